@@ -1,0 +1,209 @@
+"""Pins for the oracle's dispatch (bf16 copy, FP8 quantisation) and combine
+("GPU MoE all-to-all", section "Two collectives per layer": k copies out,
+inverse permutation back, scaled by the router's gate weights; section
+"Latency-bound at decode, bandwidth-bound at prefill": lower-precision
+dispatch; "MoE All-to-All Dispatch and Ragged Routing", section "Returning
+Tokens to the Original GPU": residual x + dx)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from combine_moe_route_07_b200.workloads import bf16_bits, bits_to_bf16
+from conftest import read_golden
+
+
+def _bf16_rand(shape, rng, scale=1.0):
+    x = torch.from_numpy((rng.standard_normal(shape) * scale).astype(np.float32))
+    return bf16_bits(x.to(torch.bfloat16))
+
+
+def _bits_to_f64(b):
+    return bits_to_bf16(b).to(torch.float64).numpy()
+
+
+def _ids(T, E, k, rng):
+    return np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+
+
+def test_dispatch_bf16_is_index_select():
+    rng = np.random.default_rng(11)
+    T, H, E, R, k = 40, 24, 8, 2, 3
+    x = _bf16_rand((T, H), rng)
+    L = oracle.layout(_ids(T, E, k, rng), E, R)
+    out = oracle.dispatch_bf16(x, L["dst_pos"], T * k)
+    ref = x[L["src_idx"] // k]          # library gather: row p <- token src/k
+    assert np.array_equal(out, ref)
+
+
+def test_dispatch_bf16_capacity_leaves_empty_rows():
+    rng = np.random.default_rng(12)
+    T, H, E, R, k, C = 30, 8, 4, 2, 2, 5
+    x = _bf16_rand((T, H), rng)
+    L = oracle.layout(_ids(T, E, k, rng), E, R, capacity=C)
+    out = oracle.dispatch_bf16(x, L["dst_pos"], E * C)
+    src = L["src_idx"]
+    assert np.array_equal(out[src >= 0], x[src[src >= 0] // k])
+    assert np.all(out[src < 0] == 0)
+
+
+def test_quantize_row_matches_torch_recipe():
+    # Library special case: torch's fp32 division for 448/amax and amax/448, an
+    # fp32 multiply and torch's float8_e4m3fn cast (nearest-even; inputs stay
+    # within +-448 so its non-saturating cast agrees with satfinite).
+    rng = np.random.default_rng(13)
+    H = 512
+    for trial in range(20):
+        x = _bf16_rand((H,), rng, scale=10.0 ** rng.integers(-3, 3))
+        q, s = oracle.quantize_row_fp8(x)
+        xf = bits_to_bf16(x).to(torch.float32).view(H // 128, 128)
+        amax = xf.abs().amax(dim=1, keepdim=True)
+        inv = torch.tensor(448.0, dtype=torch.float32) / amax
+        scaled = xf * inv
+        assert float(scaled.abs().max()) <= 448.0 * (1 + 2 ** -22)
+        scaled = scaled.clamp(-448.0, 448.0)
+        qref = scaled.to(torch.float8_e4m3fn).view(torch.uint8).reshape(-1).numpy()
+        sref = (amax / torch.tensor(448.0)).reshape(-1).numpy()
+        assert np.array_equal(q, qref)
+        assert np.array_equal(s, sref)
+
+
+def test_quantize_row_invariants():
+    rng = np.random.default_rng(14)
+    H = 256
+    x = _bf16_rand((H,), rng)
+    x[128:] = 0            # second block all zero
+    q, s = oracle.quantize_row_fp8(x)
+    assert s[1] == 0 and np.all(q[128:] == 0)
+    xf = _bits_to_f64(x)
+    blk = xf[:128]
+    i = int(np.argmax(np.abs(blk)))
+    assert q[i] & 0x7F == 0x7E              # the block's amax maps to 448
+    deq = np.array([oracle.e4m3_decode(c) for c in q[:128]]) * float(s[0])
+    # error bound: half an e4m3 quantum of the scaled value (relative 2^-4,
+    # absolute 2^-10 in the subnormal range), times the scale
+    scaled = np.abs(blk) * 448.0 / float(np.abs(blk).max())
+    bound = np.maximum(scaled * 2.0 ** -4, 2.0 ** -10) * float(s[0]) * (1 + 1e-6)
+    assert np.all(np.abs(deq - blk) <= bound + 1e-12)
+
+
+def test_dispatch_fp8_copies_codes_to_every_slot():
+    rng = np.random.default_rng(15)
+    T, H, E, R, k = 12, 256, 8, 4, 3
+    x = _bf16_rand((T, H), rng)
+    L = oracle.layout(_ids(T, E, k, rng), E, R)
+    q, s = oracle.dispatch_fp8(x, L["dst_pos"], T * k)
+    for t in range(T):
+        qr, sr = oracle.quantize_row_fp8(x[t])
+        for j in range(k):
+            p = L["dst_pos"][t, j]
+            assert np.array_equal(q[p], qr) and np.array_equal(s[p], sr)
+
+
+def test_combine_identity_experts_returns_input_exactly():
+    rng = np.random.default_rng(16)
+    T, H, E, R, k = 50, 16, 16, 4, 6
+    x = _bf16_rand((T, H), rng)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    ids, gates = oracle.route(logits, k)
+    L = oracle.layout(ids, E, R)
+    y = oracle.dispatch_bf16(x, L["dst_pos"], T * k)
+    out = oracle.combine(y, L["dst_pos"], gates, T)
+    assert np.array_equal(_bits_to_f64(out), _bits_to_f64(x))
+    # + residual: x * sum(g) + x == 2x exactly
+    out2 = oracle.combine(y, L["dst_pos"], gates, T, residual_bits=x)
+    assert np.array_equal(_bits_to_f64(out2), 2 * _bits_to_f64(x))
+
+
+def test_combine_is_nearest_bf16_of_exact_sum():
+    rng = np.random.default_rng(17)
+    T, H, E, R, k = 40, 32, 8, 2, 4
+    x = _bf16_rand((T, H), rng)
+    y = _bf16_rand((T * k, H), rng)
+    sh = _bf16_rand((T, H), rng)
+    ids = _ids(T, E, k, rng)
+    gates = rng.random((T, k)).astype(np.float32)
+    L = oracle.layout(ids, E, R)
+    out = oracle.combine(y, L["dst_pos"], gates, T, shared_bits=sh, residual_bits=x)
+    # numpy fp64 sum of the same terms (exact products, tiny summation error)
+    yf = _bits_to_f64(y)
+    exact = np.einsum("tk,tkh->th", gates.astype(np.float64), yf[L["dst_pos"]])
+    exact += _bits_to_f64(sh) + _bits_to_f64(x)
+    got = _bits_to_f64(out)
+    # nearest bf16: |got - exact| <= half a bf16 quantum of exact
+    quantum = 2.0 ** (np.floor(np.log2(np.abs(exact) + 1e-300)) - 7)
+    assert np.all(np.abs(got - exact) <= 0.5 * quantum * (1 + 1e-9))
+
+
+def test_combine_drops_contribute_nothing():
+    T, H, E, R, k, C = 6, 8, 2, 1, 2, 2
+    ids = np.tile(np.array([0, 1], np.int32), (T, 1))  # every token picks both
+    rng = np.random.default_rng(18)
+    x = _bf16_rand((T, H), rng)
+    gates = np.full((T, k), 0.5, np.float32)
+    L = oracle.layout(ids, E, R, capacity=C)
+    y = oracle.dispatch_bf16(x, L["dst_pos"], E * C)
+    out = oracle.combine(y, L["dst_pos"], gates, T, residual_bits=x)
+    xf = _bits_to_f64(x)
+    got = _bits_to_f64(out)
+    # tokens 0,1 kept both slots: 0.5x + 0.5x + x = 2x; others dropped both: x
+    assert np.array_equal(got[:2], 2 * xf[:2])
+    assert np.array_equal(got[2:], xf[2:])
+    out0 = oracle.combine(y, L["dst_pos"], gates, T)
+    assert np.all(_bits_to_f64(out0)[2:] == 0)
+
+
+def test_combine_token_subset_matches_full():
+    rng = np.random.default_rng(19)
+    T, H, E, R, k = 30, 16, 8, 2, 2
+    x = _bf16_rand((T, H), rng)
+    ids = _ids(T, E, k, rng)
+    gates = rng.random((T, k)).astype(np.float32)
+    L = oracle.layout(ids, E, R)
+    y = _bf16_rand((T * k, H), rng)
+    full = oracle.combine(y, L["dst_pos"], gates, T)
+    sub = np.array([3, 17, 29], np.int32)
+    part = oracle.combine(y, L["dst_pos"], gates, T, tokens=sub)
+    assert np.array_equal(part[sub], full[sub])
+
+
+def test_expert_scale_standin_matches_torch():
+    rng = np.random.default_rng(20)
+    T, H, E, R, k = 20, 16, 8, 2, 3
+    x = _bf16_rand((T, H), rng)
+    L = oracle.layout(_ids(T, E, k, rng), E, R)
+    xd = oracle.dispatch_bf16(x, L["dst_pos"], T * k)
+    y = oracle.expert_scale(xd, L["expert_off"], L["counts"])
+    e_of_row = np.repeat(np.arange(E), L["counts"])
+    s = (torch.arange(1, E + 1, dtype=torch.float32) / torch.tensor(float(E)))[e_of_row]
+    ref = (bits_to_bf16(xd).to(torch.float32) * s[:, None]).to(torch.bfloat16)
+    assert np.array_equal(y, bf16_bits(ref))
+
+
+def test_dequant_standin_matches_torch():
+    rng = np.random.default_rng(21)
+    q = rng.integers(0, 256, size=(7, 256), dtype=np.uint8)
+    q[(q & 0x7F) == 0x7F] = 0  # no NaN codes
+    s = (rng.random((7, 2)) * 3).astype(np.float32)
+    y = oracle.dequant_fp8(q, s)
+    qt = torch.from_numpy(q).view(torch.float8_e4m3fn).to(torch.float32)
+    ref = (qt * torch.from_numpy(s).repeat_interleave(128, dim=1)).to(torch.bfloat16)
+    assert np.array_equal(y, bf16_bits(ref))
+
+
+def test_hand_worked_combine():
+    g = read_golden("hand_route_layout.txt")
+    logits = np.array([[float(v) for v in g["logits_t0"]],
+                       [float(v) for v in g["logits_t1"]]], np.float32)
+    bias = np.array([float(v) for v in g["bias"]], np.float32)
+    x = bf16_bits(torch.tensor([[float(v) for v in g["x_t0"]],
+                                [float(v) for v in g["x_t1"]]]).to(torch.bfloat16))
+    ids, gates = oracle.route(logits, 2, bias)
+    for cap, tag in ((0, "dropless"), (1, "capacity")):
+        L = oracle.layout(ids, 4, 2, capacity=cap)
+        y = oracle.dispatch_bf16(x, L["dst_pos"], L["src_idx"].shape[0])
+        out = _bits_to_f64(oracle.combine(y, L["dst_pos"], gates, 2))
+        assert out[0].tolist() == [float(v) for v in g[f"out_{tag}_t0"]]
+        assert out[1].tolist() == [float(v) for v in g[f"out_{tag}_t1"]]
