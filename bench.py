@@ -1,0 +1,467 @@
+"""Benchmark: MoE route + layout + dispatch + combine on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill]
+    python bench.py --impl reference ...        # the CPU oracle, timed as is
+
+One step is one pass of the whole path over one batch: moe_route, moe_layout
+(count + place kernels), moe_dispatch, moe_combine.  The expert FFN between
+dispatch and combine is not part of the path; its output y (the workload's
+stand-in expert applied to a warm-up dispatch of the same batch) is prepared
+before the timed region, like the inputs.  Between timed steps a 256 MiB
+buffer is written to flush the 126 MB L2; the flush sits outside the per-step
+CUDA events, and the step time is the sum of the event intervals.
+
+Prints ONE JSON line (rank 0).  With N > 1 (torchrun, one process per GPU)
+every rank runs its own batch (weak scaling, no collective on the data path);
+the reported time is the max over ranks.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+FALLBACK_HBM_GBS = 6650.0
+METRIC = "dispatch+combine tokens/s at 1 B200; achieved HBM GB/s vs peak"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=3000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["native", "reference"], default="native")
+    p.add_argument("--workload", default="prefill")
+    p.add_argument("--e2e-steps", type=int, default=200)
+    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ------------------------------------------------------------ byte counts --
+
+def algorithmic_bytes(w, kept_rows):
+    """Bytes each step must move (SURVEY's per-token figures, summed over the
+    rows actually kept)."""
+    T, H, E, k = w.T, w.H, w.E, w.k
+    row = 2 * H
+    disp_row_out = (H + 4 * (H // 128)) if w.fp8 else row
+    b = {}
+    b["route"] = T * E * 4 + (4 * E if w.bias else 0) + T * k * 8
+    b["layout"] = T * k * 4 * 2 + T * k * 4 + w.rows * 4 + (3 * E + 2 * w.R) * 4
+    b["dispatch"] = T * row + kept_rows * disp_row_out + T * k * 4
+    b["combine"] = kept_rows * row + T * k * 8 + T * row \
+        + (T * row if w.shared else 0) + (T * row if w.residual else 0)
+    return b
+
+
+# ----------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (clocks, throttle reasons)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = None
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = []
+        self.sel = sel
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+        os.close(fd)
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *self.sel, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(self.REASONS, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ peaks --
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def ncu_traffic(kernel, workload):
+    """Per-launch DRAM bytes from the committed ncu summary, if one exists for
+    this kernel and workload (profiles/ncu_traffic.txt: `kernel workload bytes`)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    try:
+        with open(path) as f:
+            for line in f:
+                parts = line.split("#", 1)[0].split()
+                if len(parts) >= 3 and parts[0] == kernel and parts[1] == workload:
+                    return float(parts[2])
+    except OSError:
+        pass
+    return None
+
+
+# ----------------------------------------------------------------- oracle --
+
+def oracle_step_fn(w, inp, tokens):
+    """One oracle pass of the path over the first `tokens` tokens (expert
+    output prepared outside the returned closure)."""
+    import numpy as np
+    import oracle
+    from combine_moe_route_07_b200.workloads import bf16_bits
+    x = np.ascontiguousarray(bf16_bits(inp.x)[:tokens])
+    logits = np.ascontiguousarray(inp.logits.numpy()[:tokens])
+    bias = None if inp.bias is None else inp.bias.numpy()
+    cap = w.capacity if w.capacity == 0 else max(1, -(-w.capacity * tokens // w.T))
+    ids, gates = oracle.route(logits, w.k, bias, renorm=w.renorm)
+    L = oracle.layout(ids, w.E, w.R, capacity=cap, align=w.align)
+    N = L["src_idx"].shape[0]
+    if w.fp8:
+        q, s = oracle.dispatch_fp8(x, L["dst_pos"], N)
+        y = oracle.dequant_fp8(q, s)
+    else:
+        d = oracle.dispatch_bf16(x, L["dst_pos"], N)
+        y = oracle.expert_scale(d, L["expert_off"], L["counts"], cap) \
+            if w.expert == "scale" else d
+
+    def step():
+        i2, g2 = oracle.route(logits, w.k, bias, renorm=w.renorm)
+        L2 = oracle.layout(i2, w.E, w.R, capacity=cap, align=w.align)
+        if w.fp8:
+            oracle.dispatch_fp8(x, L2["dst_pos"], N)
+        else:
+            oracle.dispatch_bf16(x, L2["dst_pos"], N)
+        oracle.combine(y, L2["dst_pos"], g2, tokens, shared_bits=x if w.shared else None,
+                       residual_bits=x if w.residual else None)
+    return step
+
+
+def time_oracle(w, inp, budget_s, max_steps=None):
+    """Time the oracle on a bounded sample: the whole batch if one pass fits
+    the budget, else a prefix of tokens; returns (tokens/s, sample text)."""
+    tokens = w.T
+    step = oracle_step_fn(w, inp, tokens)
+    t0 = time.perf_counter()
+    step()
+    one = time.perf_counter() - t0
+    if one > budget_s and tokens > 1:
+        tokens = max(1, int(tokens * budget_s / one / 2))
+        step = oracle_step_fn(w, inp, tokens)
+    reps, elapsed = 0, 0.0
+    while elapsed < budget_s and (max_steps is None or reps < max_steps):
+        t0 = time.perf_counter()
+        step()
+        elapsed += time.perf_counter() - t0
+        reps += 1
+    return tokens * reps / elapsed, tokens, reps, elapsed
+
+
+def run_reference(args, w):
+    """The reference arm: the CPU oracle, as it stands, on this machine's host."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from combine_moe_route_07_b200.workloads import make_inputs
+    inp = make_inputs(w)
+    # each step is a bounded sample of the workload: a prefix of the batch
+    # sized so that the timed steps take about a minute in all
+    probe_tokens = max(1, w.T // 16)
+    step = oracle_step_fn(w, inp, probe_tokens)
+    t0 = time.perf_counter()
+    step()
+    per_token = (time.perf_counter() - t0) / probe_tokens
+    budget = 60.0 / max(1, args.steps + args.warmup)
+    tokens = int(min(w.T, max(8, budget / per_token)))
+    step = oracle_step_fn(w, inp, tokens)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = tokens * args.steps / el
+    sample = f"first {tokens} of {w.T} tokens of the {w.name} batch per step, single thread"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.describe(), "tokens_per_step": tokens},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- native --
+
+def main():
+    args = parse()
+    from combine_moe_route_07_b200.workloads import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    import combine_moe_route_07_b200 as m
+    from combine_moe_route_07_b200.workloads import make_inputs
+
+    inp = make_inputs(w, seed=w.seed + rank)
+    shape = m.MoeShape(tokens=w.T, hidden=w.H, experts=w.E, k=w.k, ranks=w.R,
+                       capacity=w.capacity, align=w.align, renorm=w.renorm, fp8=w.fp8)
+    ws = m.Workspace(shape, dev)
+    x = inp.x.to(dev)
+    logits = inp.logits.to(dev)
+    bias = None if inp.bias is None else inp.bias.to(dev)
+    T, k, N = w.T, w.k, shape.rows
+    i32 = dict(dtype=torch.int32, device=dev)
+    ids = torch.empty((T, k), **i32)
+    gates = torch.empty((T, k), dtype=torch.float32, device=dev)
+    lay = m.Layout(torch.empty(w.E, **i32), torch.empty(w.E + 1, **i32),
+                   torch.empty(w.R + 1, **i32), torch.empty(w.R, **i32),
+                   torch.empty((T, k), **i32), torch.empty(N, **i32))
+    if w.fp8:
+        xd = torch.empty((N, w.H), dtype=torch.float8_e4m3fn, device=dev)
+        sc = torch.empty((N, w.H // 128), dtype=torch.float32, device=dev)
+    else:
+        xd = torch.empty((N, w.H), dtype=torch.bfloat16, device=dev)
+        sc = None
+    out = torch.empty((T, w.H), dtype=torch.bfloat16, device=dev)
+    shared = x if w.shared else None
+    residual = x if w.residual else None
+
+    def route_layout_dispatch():
+        m.moe_route(shape, logits, bias, ws=ws, ids=ids, gates=gates)
+        m.moe_layout(shape, ids, ws=ws, out=lay)
+        m.moe_dispatch(shape, x, lay.dst_pos, ws=ws, out=xd, scales=sc)
+
+    # the expert stand-in's output for this batch, prepared once
+    route_layout_dispatch()
+    if w.fp8:
+        y = (xd.float() * sc.repeat_interleave(128, dim=1)).to(torch.bfloat16)
+    elif w.expert == "scale":
+        rows = torch.arange(N, device=dev, dtype=torch.int32)
+        e = (torch.searchsorted(lay.expert_off, rows, right=True) - 1).clamp(min=0)
+        s = (torch.arange(1, w.E + 1, dtype=torch.float32, device=dev)
+             / torch.tensor(float(w.E), device=dev))[e]
+        y = (xd.float() * s[:, None]).to(torch.bfloat16)
+    else:
+        y = xd.clone()
+    torch.cuda.synchronize()
+    kept_rows = int(lay.rank_counts.sum().item())
+    m.moe_check(ws)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    n_ev = 5  # route | layout | dispatch | combine
+    names = ("route", "layout", "dispatch", "combine")
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        m.moe_route(shape, logits, bias, ws=ws, ids=ids, gates=gates)
+        if evs is not None:
+            evs[1].record(stream)
+        m.moe_layout(shape, ids, ws=ws, out=lay)
+        if evs is not None:
+            evs[2].record(stream)
+        m.moe_dispatch(shape, x, lay.dst_pos, ws=ws, out=xd, scales=sc)
+        if evs is not None:
+            evs[3].record(stream)
+        m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared, residual=residual,
+                      out=out)
+        if evs is not None:
+            evs[4].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(K)]
+    sampler = ClockSampler(local) if rank == 0 else None
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    for i in range(K):
+        flush.fill_(1)
+        step(events[i])
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    m.moe_check(ws)
+
+    seg = [[0.0] * 4 for _ in range(K)]
+    for i in range(K):
+        for s in range(4):
+            seg[i][s] = events[i][s].elapsed_time(events[i][s + 1])  # ms
+    total_ms = sum(sum(r) for r in seg)
+    mean = [sum(seg[i][s] for i in range(K)) / K for s in range(4)]
+    if dist is not None:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # end to end through the public API: pinned host inputs in, result out
+    e2e = None
+    if args.e2e_steps > 0:
+        x_h = inp.x.pin_memory()
+        lg_h = inp.logits.pin_memory()
+        out_h = torch.empty((T, w.H), dtype=torch.bfloat16).pin_memory()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        for it in range(3 + args.e2e_steps):
+            if it == 3:
+                torch.cuda.synchronize()
+                e0.record(stream)
+            x.copy_(x_h, non_blocking=True)
+            logits.copy_(lg_h, non_blocking=True)
+            step()
+            out_h.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        if dist is not None:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": x_h.numel() * 2 + lg_h.numel() * 4,
+               "d2h_bytes_per_step": out_h.numel() * 2, "ms_per_step": e2e_ms}
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return 0
+
+    byts = algorithmic_bytes(w, kept_rows)
+    peak, peak_kind = hbm_peak()
+    kern = {}
+    for s, name in enumerate(names):
+        us = mean[s] * 1e3
+        gbs = byts[name] / (mean[s] * 1e-3) / 1e9
+        kern[name] = {"us": round(us, 2), "bytes": byts[name], "gbs": round(gbs, 1),
+                      "frac": round(gbs / peak, 4)}
+    dom = "dispatch" if mean[2] >= mean[3] else "combine"
+    dom_gbs = byts[dom] / (mean[names.index(dom)] * 1e-3) / 1e9
+    dc_ms = mean[2] + mean[3]
+    dc_gbs = (byts["dispatch"] + byts["combine"]) / (dc_ms * 1e-3) / 1e9
+    ms_step = total_ms / K
+    line = {
+        "metric": METRIC,
+        "value": world * T * K / (total_ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8-e4m3 dispatch, bf16 rows, fp32 accumulate" if w.fp8 else "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.describe(), "tokens": T, "hidden": w.H, "experts": w.E,
+                   "k": k, "ranks": w.R, "capacity": w.capacity, "rows": N,
+                   "kept_rows": kept_rows, "parallelism": f"replicas x{world}",
+                   "l2": "256 MiB write between timed steps, outside the step events",
+                   "step": "route + layout(count, place) + dispatch + combine"},
+        "dispatch_combine": {"tokens_per_s": world * T / (dc_ms * 1e-3),
+                             "us": round(dc_ms * 1e3, 2), "gbs": round(dc_gbs, 1),
+                             "frac": round(dc_gbs / peak, 4),
+                             "frac_of_8tbs": round(dc_gbs / 8000.0, 4)},
+        "kernels": kern,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(dom_gbs, 1),
+                     "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
+                     "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
+                     "traffic": ncu_traffic(dom, w.name)},
+        "gpu_launches": 5 * K,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        v, tokens, reps, el = time_oracle(w, inp, args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{reps} single-threaded oracle passes over the first {tokens} of "
+                      f"{T} tokens of the same batch ({el:.1f} s)"}
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

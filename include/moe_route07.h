@@ -1,0 +1,188 @@
+/*
+ * moe_route07.h -- C ABI of the on-GPU MoE token route / layout / dispatch /
+ * combine path (NVIDIA B200, sm_100a).
+ *
+ * The four steps are the data-parallel part of the expert-parallel exchange
+ * that the following pages describe:
+ *   "GPU MoE all-to-all" (aicassindra): section "Two collectives per layer,
+ *      and what each one moves" (dispatch replicates each token to its k
+ *      experts, combine is the inverse permutation scaled by the gate weights,
+ *      per-destination counts travel before the payload) and section
+ *      "Bucketing: cut the message count, not the byte count" (sort rows by
+ *      destination, build the offset table, keep counts on the device);
+ *   "19. All-to-all" (ai-from-scratch): section "Why the router can ruin your
+ *      day" (a per-expert bias used only for the top-k decision; tokens over
+ *      capacity are dropped as if they skipped the expert);
+ *   "MoE All-to-All Dispatch and Ragged Routing": section "Fixed Capacity vs.
+ *      Ragged Routing" (capacity factor with drops, or dropless ragged
+ *      layout) and section "Returning Tokens to the Original GPU" (x + dx);
+ *   "Mixture-of-experts acceleration through overlap" (thecoregrid): the
+ *      remote-owner-aligned layout (every row band bound to one destination).
+ *
+ * Everything runs on one GPU.  The R "ranks" are logical partitions of the
+ * dispatched buffer: expert e belongs to rank e / (E/R), and each rank's rows
+ * form one contiguous slice.
+ *
+ * Conventions for every call:
+ *  - All pointers except `shape` are DEVICE pointers owned by the caller; the
+ *    library allocates nothing and keeps no state between calls.
+ *  - Calls are asynchronous on `stream` (NULL = legacy default stream).  Only
+ *    moe_get_device_error synchronises.
+ *  - Arguments are checked on the host first; on MOE_ERR_INVALID_ARG nothing
+ *    is launched and no buffer is touched.
+ *  - Problems found by the kernels (an expert id or row outside its range, a
+ *    NaN routing key, a wait that gave up) never trap: the kernel records the
+ *    first one in the workspace's error word and skips the offending element.
+ *    moe_get_device_error reads and clears it.
+ *  - A launch failure returns MOE_ERR_CUDA.
+ *  - One workspace serves one stream at a time; calls that share a workspace
+ *    must be ordered on the device (same stream, or event-ordered).
+ */
+#ifndef MOE_ROUTE07_H
+#define MOE_ROUTE07_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,    /* host check failed; nothing launched */
+  MOE_ERR_UNSUPPORTED = 2,    /* valid request outside what this build covers */
+  MOE_ERR_WORKSPACE = 3,      /* workspace NULL, misaligned or too small */
+  MOE_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
+  MOE_ERR_DEVICE_RANGE = 5,   /* device: expert id or row index out of range */
+  MOE_ERR_DEVICE_TIMEOUT = 6, /* device: a bounded wait in moe_layout gave up */
+  MOE_ERR_DEVICE_NAN = 7      /* device: a routing key was NaN */
+} moe_status_t;
+
+/* flags */
+#define MOE_F_RENORM 0x1u /* gates: softmax over the k selected experts (else over all E) */
+#define MOE_F_FP8 0x2u    /* dispatch writes e4m3 codes + per-128-channel fp32 scales */
+
+/* Problem description (host memory).
+ *   tokens   T >= 0
+ *   hidden   H, multiple of 8 (bf16 rows of 16-byte multiples); multiple of
+ *            128 with MOE_F_FP8
+ *   experts  E, 1..1024, multiple of ranks
+ *   k        slots per token, 1..min(E, 32)
+ *   ranks    R >= 1 logical EP ranks (E/R consecutive experts each)
+ *   capacity 0: dropless; C > 0: every expert owns exactly C rows and keeps
+ *            its first C assignments in token order
+ *   align    >= 1: dropless segments are rounded up to a multiple of align
+ *            rows (must be 1 in capacity mode)
+ *   flags    MOE_F_* bits
+ * Limits: T*k < 2^30, and the layout's row count below 2^31. */
+typedef struct {
+  int32_t tokens, hidden, experts, k, ranks;
+  int32_t capacity;
+  int32_t align;
+  uint32_t flags;
+} moe_shape_t;
+
+/* Rows N of the dispatched buffer: dropless T*k + E*(align-1), capacity E*C.
+ * A static bound, so buffers are sized without reading counts back.
+ * Returns -1 for an invalid shape. */
+int64_t moe_layout_rows(const moe_shape_t* shape);
+
+/* Bytes of device workspace the calls need for `shape` (error word, block
+ * ticket and the layout's per-block prefix table).  0 for an invalid shape.
+ * A workspace sized for one shape serves any shape whose requirement is not
+ * larger. */
+size_t moe_workspace_bytes(const moe_shape_t* shape);
+
+/* Zero-fill a workspace (cudaMemsetAsync on `stream`).  Required once before
+ * the workspace's first use; every call leaves it ready for the next one. */
+moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Step 1 -- route ("19. All-to-all", section "Why the router can ruin your
+ * day").  For each token t:
+ *   key[e]   = logits[t,e] + bias[e]       (one fp32 add; bias NULL = 0)
+ *   ids[t,j] = the expert with the j-th largest key; equal keys (+0 == -0)
+ *              order by the lower expert id
+ *   gates[t,j] = softmax of the RAW logits (the bias never enters the mix
+ *              weights) over the k selected experts with MOE_F_RENORM, else
+ *              over all E experts read at the selected ones.
+ * logits fp32 [T,E] row-major; bias fp32 [E] or NULL; ids int32 [T,k];
+ * gates fp32 [T,k].  All 4-byte aligned.  A NaN key sets MOE_ERR_DEVICE_NAN.
+ */
+moe_status_t moe_route(const moe_shape_t* shape, const float* logits, const float* bias,
+                       int32_t* ids, float* gates, void* ws, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/* Steps 2 and 3 -- count histogram and layout scan ("GPU MoE all-to-all",
+ * sections "Two collectives per layer" and "Bucketing"; "MoE All-to-All
+ * Dispatch and Ragged Routing", section "Fixed Capacity vs. Ragged Routing").
+ *   ids         int32 [T,k] expert ids (from moe_route or the caller)
+ *   counts      int32 [E]   assignments per expert, before any drop
+ *   expert_off  int32 [E+1] first row of each expert's segment; [E] = rows used
+ *   rank_off    int32 [R+1] first row of each rank's slice; [R] = rows used
+ *   rank_counts int32 [R]   rows of each rank's slice that hold a token -- the
+ *                           per-destination counts an exchange posts first
+ *   dst_pos     int32 [T,k] row of assignment (t,j); -1 if dropped
+ *   src_idx     int32 [N]   t*k+j of the assignment in each row; -1 if empty
+ * Within an expert, rows follow token order; in capacity mode the first C
+ * assignments in that order are kept.  Results are deterministic: no output
+ * depends on block scheduling.  An id outside [0,E) sets
+ * MOE_ERR_DEVICE_RANGE and that assignment is treated as dropped. */
+moe_status_t moe_layout(const moe_shape_t* shape, const int32_t* ids, int32_t* counts,
+                        int32_t* expert_off, int32_t* rank_off, int32_t* rank_counts,
+                        int32_t* dst_pos, int32_t* src_idx, void* ws, size_t ws_bytes,
+                        moe_stream_t stream);
+
+/* Step 4 -- dispatch ("GPU MoE all-to-all", sections "Bucketing" and
+ * "Latency-bound at decode, bandwidth-bound at prefill").
+ *   x       bf16 [T,H], 16-byte aligned
+ *   dst_pos int32 [T,k] from moe_layout
+ *   out     bf16 [N,H] (or e4m3 [N,H] with MOE_F_FP8), 16-byte aligned:
+ *           row dst_pos[t,j] receives token t.  Rows no assignment maps to
+ *           are not written.
+ *   scales  fp32 [N,H/128] with MOE_F_FP8 (else ignored, may be NULL):
+ *           per 128-channel block b of token t, amax = max|x|,
+ *           scale = amax/448, codes = e4m3_rn_satfinite(x * (448/amax));
+ *           amax == 0 gives codes 0 and scale 0.
+ * A dst_pos value >= N sets MOE_ERR_DEVICE_RANGE and that copy is skipped. */
+moe_status_t moe_dispatch(const moe_shape_t* shape, const void* x, const int32_t* dst_pos,
+                          void* out, float* scales, void* ws, size_t ws_bytes,
+                          moe_stream_t stream);
+
+/* Step 5 -- combine ("GPU MoE all-to-all", section "Two collectives per
+ * layer": the inverse permutation scaled by the router's gate weights; "MoE
+ * All-to-All Dispatch and Ragged Routing", section "Returning Tokens to the
+ * Original GPU": the residual x + dx).
+ *   out[t,c] = bf16_rn( sum_{j, dst_pos[t,j] >= 0} gates[t,j] * y[dst_pos[t,j], c]
+ *                       + shared[t,c] + residual[t,c] )
+ * accumulated in fp32 in slot order j = 0..k-1, then shared, then residual.
+ *   y        bf16 [N,H] expert outputs in the layout's row order
+ *   shared   bf16 [T,H] always-on expert output, or NULL
+ *   residual bf16 [T,H] the layer input x, or NULL
+ *   out      bf16 [T,H]
+ * bf16 buffers 16-byte aligned.  A dropped slot contributes nothing; the other
+ * gates are not rescaled. */
+moe_status_t moe_combine(const moe_shape_t* shape, const void* y, const int32_t* dst_pos,
+                         const float* gates, const void* shared, const void* residual,
+                         void* out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Synchronise `stream`, return the first device-side error recorded in `ws`
+ * since the last read (MOE_OK if none) and clear it.  *detail (may be NULL)
+ * receives the offending index (expert id, row, or block) when known. */
+moe_status_t moe_get_device_error(void* ws, int32_t* detail, moe_stream_t stream);
+
+/* Static description of a status code. */
+const char* moe_status_string(moe_status_t status);
+
+/* ABI version of this header (bumped on any incompatible change). */
+#define MOE_ABI_VERSION 1
+int32_t moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_ROUTE07_H */

@@ -1,0 +1,190 @@
+"""Test helpers: run the CUDA path (through the C ABI binding) and the CPU
+oracle on the same seeded inputs, plus comparison helpers.
+
+The expert FFN is outside the path; between dispatch and combine both sides
+apply the same stand-in expert (identity, "row of expert e times (e+1)/E", or
+FP8 dequantisation).  On the GPU side the stand-in uses plain torch ops; on
+the oracle side the oracle's own stand-in functions.
+"""
+import functools
+
+import numpy as np
+import torch
+
+import oracle
+from combine_moe_route_07_b200.workloads import (WORKLOADS, Workload, bf16_bits, bits_to_bf16,
+                                                 make_inputs)
+
+
+@functools.lru_cache(maxsize=2)
+def _inputs_cached(T, H, E, zipf_s, bias, seed):
+    w = Workload("tmp", T=T, H=H, E=E, R=1, k=1, zipf_s=zipf_s, bias=bias, seed=seed)
+    return make_inputs(w)
+
+
+def inputs_for(w: Workload):
+    return _inputs_cached(w.T, w.H, w.E, w.zipf_s, w.bias, w.seed)
+
+
+def shape_of(w: Workload):
+    from combine_moe_route_07_b200 import MoeShape
+    return MoeShape(tokens=w.T, hidden=w.H, experts=w.E, k=w.k, ranks=w.R, capacity=w.capacity,
+                    align=w.align, renorm=w.renorm, fp8=w.fp8)
+
+
+# ------------------------------------------------------------- stand-ins ----
+
+def row_expert(expert_off: torch.Tensor, N: int) -> torch.Tensor:
+    rows = torch.arange(N, device=expert_off.device, dtype=torch.int32)
+    return (torch.searchsorted(expert_off, rows, right=True) - 1).clamp(min=0)
+
+
+def standin_gpu(w: Workload, dispatched, lay):
+    if w.expert == "identity":
+        return dispatched
+    if w.expert == "scale":
+        e = row_expert(lay.expert_off, dispatched.shape[0])
+        s = (torch.arange(1, w.E + 1, dtype=torch.float32, device=e.device)
+             / torch.tensor(float(w.E), device=e.device))[e]
+        return (dispatched.float() * s[:, None]).to(torch.bfloat16)
+    if w.expert == "dequant":
+        q, sc = dispatched
+        return (q.float() * sc.repeat_interleave(128, dim=1)).to(torch.bfloat16)
+    raise ValueError(w.expert)
+
+
+def standin_oracle(w: Workload, disp, L):
+    if w.expert == "identity":
+        return disp
+    if w.expert == "scale":
+        return oracle.expert_scale(disp, L["expert_off"], L["counts"], w.capacity)
+    if w.expert == "dequant":
+        q, s = disp
+        return oracle.dequant_fp8(q, s)
+    raise ValueError(w.expert)
+
+
+# ------------------------------------------------------------ the paths ----
+
+def run_gpu(w: Workload, inp, ids=None, gates=None):
+    """Run route (unless ids/gates are given), layout, dispatch, stand-in and
+    combine on cuda:0.  Returns a dict of CUDA tensors and the workspace."""
+    import combine_moe_route_07_b200 as m
+    dev = torch.device("cuda:0")
+    shape = shape_of(w)
+    ws = m.Workspace(shape, dev)
+    x = inp.x.to(dev)
+    res = {"ws": ws, "x": x}
+    if ids is None:
+        logits = inp.logits.to(dev)
+        bias = None if inp.bias is None else inp.bias.to(dev)
+        ids, gates = m.moe_route(shape, logits, bias, ws=ws)
+    else:
+        ids = torch.from_numpy(np.ascontiguousarray(ids)).to(dev)
+        gates = torch.from_numpy(np.ascontiguousarray(gates)).to(dev)
+    res["ids"], res["gates"] = ids, gates
+    lay = m.moe_layout(shape, ids, ws=ws)
+    res["layout"] = lay
+    disp = m.moe_dispatch(shape, x, lay.dst_pos, ws=ws)
+    res["dispatch"] = disp
+    y = standin_gpu(w, disp, lay)
+    res["y"] = y
+    res["out"] = m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws,
+                               shared=x if w.shared else None,
+                               residual=x if w.residual else None)
+    torch.cuda.synchronize()
+    return res
+
+
+def run_oracle(w: Workload, inp, through="combine"):
+    """The oracle's whole path on the host (numpy)."""
+    x = bf16_bits(inp.x)
+    logits = inp.logits.numpy()
+    bias = None if inp.bias is None else inp.bias.numpy()
+    ids, gates = oracle.route(logits, w.k, bias, renorm=w.renorm)
+    res = {"ids": ids, "gates": gates, "x": x}
+    if through == "route":
+        return res
+    L = oracle.layout(ids, w.E, w.R, capacity=w.capacity, align=w.align)
+    res["layout"] = L
+    if through == "layout":
+        return res
+    N = L["src_idx"].shape[0]
+    disp = oracle.dispatch_fp8(x, L["dst_pos"], N) if w.fp8 else oracle.dispatch_bf16(
+        x, L["dst_pos"], N)
+    res["dispatch"] = disp
+    y = standin_oracle(w, disp, L)
+    res["y"] = y
+    res["out"] = oracle.combine(y, L["dst_pos"], gates, w.T,
+                                shared_bits=x if w.shared else None,
+                                residual_bits=x if w.residual else None)
+    return res
+
+
+def oracle_combine_sampled(w: Workload, x_bits, ids, gates, dst_pos, tokens):
+    """Oracle combine for a sample of tokens, building only those tokens'
+    expert outputs (each token's k rows are its own dispatched copies)."""
+    tokens = np.asarray(tokens, np.int32)
+    n, k = len(tokens), w.k
+    xs = x_bits[tokens]
+    dp = dst_pos[tokens]
+    local = np.where(dp >= 0, np.arange(n * k, dtype=np.int32).reshape(n, k), -1).astype(np.int32)
+    if w.fp8:
+        q, s = oracle.dispatch_fp8(xs, local, n * k)
+        y = oracle.dequant_fp8(q, s)
+    else:
+        y = oracle.dispatch_bf16(xs, local, n * k)
+        if w.expert == "scale":
+            y = _scale_rows(w, y, ids[tokens].reshape(-1).astype(np.int32))
+    out = oracle.combine(y, local, gates[tokens], n,
+                         shared_bits=xs if w.shared else None,
+                         residual_bits=xs if w.residual else None)
+    return out
+
+
+def _scale_rows(w, y, e_of_row):
+    """oracle.expert_scale on rows whose experts are given one by one."""
+    out = y.copy()
+    for e in np.unique(e_of_row):
+        rows = np.nonzero(e_of_row == e)[0]
+        counts = np.zeros(w.E, np.int32)
+        counts[e] = len(rows)
+        off = np.zeros(w.E + 1, np.int32)
+        off[e + 1:] = len(rows)
+        out[rows] = oracle.expert_scale(y[rows], off, counts)
+    return out
+
+
+# ------------------------------------------------------------ comparisons --
+
+def to_np(t: torch.Tensor):
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy()
+    return t.numpy()
+
+
+def bf16_ulp_diff(a_bits, b_bits):
+    """|ordered(a) - ordered(b)| for bf16 bit patterns (+0 and -0 coincide)."""
+    def ordered(v):
+        v = v.astype(np.int32)
+        mag = v & 0x7FFF
+        return np.where(v & 0x8000, -mag, mag)
+    return np.abs(ordered(np.asarray(a_bits)) - ordered(np.asarray(b_bits)))
+
+
+def assert_bf16_close(got_bits, want_bits, ulps=1, what=""):
+    d = bf16_ulp_diff(got_bits, want_bits)
+    bad = int((d > ulps).sum())
+    assert bad == 0, f"{what}: {bad} of {d.size} values differ by more than {ulps} bf16 ulp " \
+                     f"(max {int(d.max())})"
+    return d
+
+
+def assert_gates_close(got, want, rel=1e-6, what="gates"):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    err = np.abs(got - want) / np.maximum(np.abs(want), 1e-300)
+    assert float(err.max(initial=0.0)) <= rel, f"{what}: max relative error {err.max()}"

@@ -1,0 +1,139 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.
+
+Tolerances (from the arithmetic, stated once here):
+  ids, counts, offsets, dst_pos, src_idx, dispatched bf16 rows, e4m3 codes and
+  fp32 scales: bit-exact (integer work, copies, and fp32 decisions taken in the
+  same precision on both sides);
+  gates: 1e-6 relative (GPU fp64 softmax rounded once vs the oracle's fp64);
+  combine: 1 bf16 ulp (GPU fp32 slot-order FMAs vs the oracle's fp64 sum, both
+  rounded once to bf16; the fp32 error is far below half a bf16 ulp, so only
+  values next to a rounding midpoint can land one ulp apart).
+"""
+import numpy as np
+import pytest
+import torch
+
+from combine_moe_route_07_b200.workloads import WORKLOADS
+from pipeline import (assert_bf16_close, assert_gates_close, inputs_for, oracle_combine_sampled,
+                      run_gpu, run_oracle, to_np)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = ["tiny", "prefill", "decode"]
+BIG = ["skewed_capacity", "skewed_dropless", "finegrained"]
+LAYOUT_KEYS = ("counts", "expert_off", "rank_off", "rank_counts", "dst_pos", "src_idx")
+
+
+def _compare_layout(g_lay, L, what):
+    for key in LAYOUT_KEYS:
+        got = to_np(getattr(g_lay, key))
+        assert np.array_equal(got, L[key]), f"{what}: layout.{key} differs"
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_full_path_small_configs(name):
+    w = WORKLOADS[name]
+    inp = inputs_for(w)
+    o = run_oracle(w, inp)
+    g = run_gpu(w, inp)
+    import combine_moe_route_07_b200 as m
+    assert m.moe_get_device_error(g["ws"]) == (0, 0)
+    assert np.array_equal(to_np(g["ids"]), o["ids"])
+    assert_gates_close(to_np(g["gates"]), o["gates"])
+    _compare_layout(g["layout"], o["layout"], name)
+    assert np.array_equal(to_np(g["dispatch"]), o["dispatch"])
+    assert_bf16_close(to_np(g["out"]), o["out"], 1, name)
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_each_kernel_on_oracle_inputs(name):
+    """Feed the oracle's intermediates to the GPU path so each kernel is
+    checked on its own (layout on the oracle's ids, combine on the oracle's
+    expert outputs and gates)."""
+    import combine_moe_route_07_b200 as m
+    from pipeline import shape_of
+    w = WORKLOADS[name]
+    inp = inputs_for(w)
+    o = run_oracle(w, inp)
+    g = run_gpu(w, inp, ids=o["ids"], gates=o["gates"])
+    _compare_layout(g["layout"], o["layout"], name)
+    shape = shape_of(w)
+    dev = g["x"].device
+    y = torch.from_numpy(o["y"].view(np.int16)).view(torch.bfloat16).to(dev)
+    dst = torch.from_numpy(o["layout"]["dst_pos"]).to(dev)
+    gates = torch.from_numpy(o["gates"]).to(dev)
+    out = m.moe_combine(shape, y, dst, gates, ws=g["ws"],
+                        shared=g["x"] if w.shared else None,
+                        residual=g["x"] if w.residual else None)
+    d = assert_bf16_close(to_np(out), o["out"], 1, name)
+    # the 1-ulp cases are rare: the fp32 path agrees almost everywhere
+    assert (d == 0).mean() > 0.999
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", BIG)
+def test_full_size_route_layout_exact_and_sampled_payload(name):
+    import combine_moe_route_07_b200 as m
+    w = WORKLOADS[name]
+    inp = inputs_for(w)
+    o = run_oracle(w, inp, through="layout")
+    g = run_gpu(w, inp)
+    assert m.moe_get_device_error(g["ws"]) == (0, 0)
+    assert np.array_equal(to_np(g["ids"]), o["ids"])
+    assert_gates_close(to_np(g["gates"]), o["gates"])
+    _compare_layout(g["layout"], o["layout"], name)
+
+    dst = o["layout"]["dst_pos"]
+    rng = np.random.default_rng(123)
+    tokens = np.unique(np.concatenate([rng.choice(w.T, 384, replace=False),
+                                       [0, 1, w.T - 1]])).astype(np.int32)
+    x = o["x"]
+    # dispatch: sampled rows against the oracle, one token at a time
+    if w.fp8:
+        import oracle
+        rows = dst[tokens]
+        idx = torch.from_numpy(rows.reshape(-1)).long().to(g["x"].device)
+        q_got = to_np(g["dispatch"][0][idx]).reshape(len(tokens), w.k, w.H)
+        s_got = to_np(g["dispatch"][1][idx]).reshape(len(tokens), w.k, w.H // 128)
+        for n, t in enumerate(tokens):
+            q, s = oracle.quantize_row_fp8(x[t])
+            for j in range(w.k):
+                assert np.array_equal(q_got[n, j], q), (t, j)
+                assert np.array_equal(s_got[n, j], s), (t, j)
+    else:
+        rows = dst[tokens]
+        keep = rows >= 0
+        got = to_np(g["dispatch"][torch.from_numpy(rows[keep]).long().to(g["x"].device)])
+        want = np.repeat(x[tokens], w.k, axis=0)[keep.reshape(-1)]
+        assert np.array_equal(got, want)
+        # property at full size: every kept copy equals its source row
+        dp = g["layout"].dst_pos
+        kept = dp >= 0
+        src_tok = torch.arange(w.T, device=dp.device)[:, None].expand_as(dp)[kept]
+        assert torch.equal(g["dispatch"][dp[kept].long()], g["x"][src_tok])
+    # combine: sampled tokens against the oracle
+    want = oracle_combine_sampled(w, x, o["ids"], o["gates"], dst, tokens)
+    got = to_np(g["out"])[tokens]
+    assert_bf16_close(got, want, 1, name)
+
+
+def test_layout_is_deterministic_under_contention():
+    import combine_moe_route_07_b200 as m
+    from pipeline import shape_of
+    w = WORKLOADS["skewed_dropless"].with_(T=8192)
+    inp = inputs_for(WORKLOADS["skewed_dropless"])
+    dev = torch.device("cuda:0")
+    shape = shape_of(w)
+    ws = m.Workspace(shape, dev)
+    logits = inp.logits[: w.T].contiguous().to(dev)
+    ids, _ = m.moe_route(shape, logits, None, ws=ws)
+    a = m.moe_layout(shape, ids, ws=ws)
+    outs = [[to_np(getattr(a, key)) for key in LAYOUT_KEYS]]
+    for _ in range(3):
+        b = m.moe_layout(shape, ids, ws=ws)
+        outs.append([to_np(getattr(b, key)) for key in LAYOUT_KEYS])
+    for other in outs[1:]:
+        for u, v in zip(outs[0], other):
+            assert np.array_equal(u, v)
+    assert m.moe_get_device_error(ws) == (0, 0)
