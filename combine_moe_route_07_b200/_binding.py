@@ -27,7 +27,7 @@ MOE_F_FP8 = 0x2
 EXPORTS = (
     "moe_abi_version", "moe_status_string", "moe_layout_rows", "moe_workspace_bytes",
     "moe_workspace_init", "moe_route", "moe_layout", "moe_dispatch", "moe_combine",
-    "moe_get_device_error",
+    "moe_get_device_error", "moe_layout_noalloc",
 )
 
 
@@ -76,6 +76,8 @@ def lib(path: str = None):
     L.moe_dispatch.restype = i32
     L.moe_combine.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.moe_combine.restype = i32
+    L.moe_layout_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.moe_layout_noalloc.restype = i32
     L.moe_get_device_error.argtypes = [vp, ctypes.POINTER(i32), vp]
     L.moe_get_device_error.restype = i32
     if path is None:

@@ -1,0 +1,101 @@
+// layout_noalloc.cu -- moe_layout for callers that cannot allocate device
+// memory.
+//
+// Some callers have no way to hand the library a workspace: plugin or
+// custom-op hosts that pass a kernel only its inputs and outputs, serving
+// runtimes whose memory pool owns every byte of the device, and code on a
+// latency-critical path where cudaMalloc (which may synchronise the device)
+// is not allowed.  This entry point runs the same count and place kernels as
+// moe_layout, with their scratch (error word, block ticket and the per-tile
+// prefix table) in a file-scope device array instead of a caller workspace.
+//
+// The array is kMoeNoallocScratchBytes bytes; every GPU that loads the library
+// holds it until the process exits.  The first call on a device looks up its
+// device address (cudaGetSymbolAddress, with that device current) and clears
+// it; make that first call before any stream capture.  Each call then clears
+// the header (error word and ticket) on the caller's stream.  Calls share the
+// array, so calls that overlap on the GPU (different streams, or different
+// host threads, without ordering) race and give wrong results.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "moe_route07.h"
+
+namespace {
+
+constexpr size_t kHeader = sizeof(moe::WsHeader);
+constexpr size_t kMoeNoallocScratchBytes = kHeader + MOE_NOALLOC_TABLE_BYTES;
+
+static __device__ __align__(256) unsigned char g_layout_scratch[kMoeNoallocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_scratch_ptr[kMaxDevices] = {nullptr};
+std::mutex g_scratch_mu;
+
+// Device address of the scratch array on the current device; the first call
+// per device resolves it and zero-fills the array.
+moe_status_t scratch_for_current_device(cudaStream_t stream, void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_layout_scratch) != cudaSuccess || p == nullptr)
+      return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(p, 0, kMoeNoallocScratchBytes, stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" moe_status_t moe_layout_noalloc(const moe_shape_t* shape, const int32_t* ids,
+                                           int32_t* counts, int32_t* expert_off,
+                                           int32_t* rank_off, int32_t* rank_counts,
+                                           int32_t* dst_pos, int32_t* src_idx,
+                                           moe_stream_t stream) {
+  // Shape checks: the same limits as moe_layout, plus the static table size.
+  const int64_t rows = moe_layout_rows(shape);
+  if (rows < 0) return MOE_ERR_INVALID_ARG;
+  const size_t need = moe_workspace_bytes(shape);
+  if (need == 0) return MOE_ERR_INVALID_ARG;
+  if (need > kMoeNoallocScratchBytes) return MOE_ERR_UNSUPPORTED;
+  if (counts == nullptr || expert_off == nullptr || rank_off == nullptr ||
+      rank_counts == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (shape->tokens > 0 && (ids == nullptr || dst_pos == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (rows > 0 && src_idx == nullptr) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {ids, counts, expert_off, rank_off, rank_counts, dst_pos, src_idx};
+  for (const void* p : ptrs)
+    if ((reinterpret_cast<uintptr_t>(p) & 3u) != 0u) return MOE_ERR_INVALID_ARG;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  void* scratch = nullptr;
+  moe_status_t st = scratch_for_current_device(s, &scratch);
+  if (st != MOE_OK) return st;
+  // error word and ticket start at zero for every call
+  if (cudaMemsetAsync(scratch, 0, kHeader, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  moe::LaunchEnv env;
+  env.stream = s;
+  env.num_sms = sms;
+  moe::WsHeader* hdr = static_cast<moe::WsHeader*>(scratch);
+  uint32_t* table = reinterpret_cast<uint32_t*>(static_cast<char*>(scratch) + kHeader);
+  const cudaError_t err = moe::launch_layout(
+      env, ids, shape->tokens, shape->experts, shape->k, shape->ranks, shape->capacity,
+      shape->align, rows, table, hdr, counts, expert_off, rank_off, rank_counts, dst_pos,
+      src_idx, 1000000000ull);
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}

@@ -169,6 +169,33 @@ moe_status_t moe_combine(const moe_shape_t* shape, const void* y, const int32_t*
                          const float* gates, const void* shared, const void* residual,
                          void* out, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_layout without a workspace, for callers that cannot allocate device
+ * memory: plugin or custom-op hosts that give a kernel only its inputs and
+ * outputs, serving runtimes whose pool owns all device memory, and
+ * latency-critical code that may not call cudaMalloc (it can synchronise the
+ * device).  The pages have no counterpart to this call; it is an interface
+ * convenience.
+ *
+ * Same arguments, results and determinism as moe_layout, minus `ws`.  The
+ * scratch lives in a static device array of 256 + MOE_NOALLOC_TABLE_BYTES
+ * bytes that every GPU loading the library keeps until the process exits.
+ * Limit: ceil(T / 128) * E * 4 <= MOE_NOALLOC_TABLE_BYTES, i.e.
+ * ceil(T/128) * E <= 524288 (T = 65536 with E = 1024, T = 131072 with
+ * E = 512); larger shapes return MOE_ERR_UNSUPPORTED and launch nothing.
+ * Allocates nothing: no cudaMalloc / cudaFree or allocating library call.
+ *  - The first call on a device resolves the array's device address and
+ *    zero-fills it (cudaMemsetAsync on `stream`): make that first call before
+ *    any stream capture.
+ *  - Every call clears the scratch header on `stream` before its kernels.
+ *  - All calls share the one array, so calls that overlap on the GPU race;
+ *    order them (one stream, or events).
+ *  - Device-side problems are not reported (there is no workspace to read
+ *    them from); an id outside [0,E) still comes out as dst_pos -1. */
+#define MOE_NOALLOC_TABLE_BYTES (2u << 20)
+moe_status_t moe_layout_noalloc(const moe_shape_t* shape, const int32_t* ids, int32_t* counts,
+                                int32_t* expert_off, int32_t* rank_off, int32_t* rank_counts,
+                                int32_t* dst_pos, int32_t* src_idx, moe_stream_t stream);
+
 /* Synchronise `stream`, return the first device-side error recorded in `ws`
  * since the last read (MOE_OK if none) and clear it.  *detail (may be NULL)
  * receives the offending index (expert id, row, or block) when known. */
