@@ -42,6 +42,8 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=200)
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--path", choices=["fused", "separate"], default="fused",
+                   help="route+layout as one moe_route_layout call, or two calls")
     return p.parse_args()
 
 
@@ -55,10 +57,12 @@ def algorithmic_bytes(w, kept_rows):
     disp_row_out = (H + 4 * (H // 128)) if w.fp8 else row
     b = {}
     b["route"] = T * E * 4 + (4 * E if w.bias else 0) + T * k * 8
-    b["layout"] = T * k * 4 * 2 + T * k * 4 + w.rows * 4 + (3 * E + 2 * w.R) * 4
+    b["layout"] = T * k * 4 * 2 + w.rows * 4 + (3 * E + 2 * w.R) * 4  # ids in, dst_pos/src_idx out
     b["dispatch"] = T * row + kept_rows * disp_row_out + T * k * 4
     b["combine"] = kept_rows * row + T * k * 8 + T * row \
         + (T * row if w.shared else 0) + (T * row if w.residual else 0)
+    # fused route + layout: the ids stay in the CTA between the two steps
+    b["route_layout"] = b["route"] + b["layout"] - T * k * 4
     return b
 
 
@@ -320,33 +324,53 @@ def main():
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    n_ev = 5  # route | layout | dispatch | combine
-    names = ("route", "layout", "dispatch", "combine")
 
-    def step(evs=None):
-        if evs is not None:
-            evs[0].record(stream)
-        m.moe_route(shape, logits, bias, ws=ws, ids=ids, gates=gates)
-        if evs is not None:
-            evs[1].record(stream)
-        m.moe_layout(shape, ids, ws=ws, out=lay)
-        if evs is not None:
-            evs[2].record(stream)
-        m.moe_dispatch(shape, x, lay.dst_pos, ws=ws, out=xd, scales=sc)
-        if evs is not None:
-            evs[3].record(stream)
-        m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared, residual=residual,
-                      out=out)
-        if evs is not None:
-            evs[4].record(stream)
+    if args.path == "fused":
+        names = ("route_layout", "dispatch", "combine")
+        ops = (
+            lambda: m.moe_route_layout(shape, logits, bias, ws=ws, ids=ids, gates=gates,
+                                       out=lay),
+            lambda: m.moe_dispatch(shape, x, lay.dst_pos, ws=ws, out=xd, scales=sc),
+            lambda: m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared,
+                                  residual=residual, out=out),
+        )
+    else:
+        names = ("route", "layout", "dispatch", "combine")
+        ops = (
+            lambda: m.moe_route(shape, logits, bias, ws=ws, ids=ids, gates=gates),
+            lambda: m.moe_layout(shape, ids, ws=ws, out=lay),
+            lambda: m.moe_dispatch(shape, x, lay.dst_pos, ws=ws, out=xd, scales=sc),
+            lambda: m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared,
+                                  residual=residual, out=out),
+        )
 
-    for _ in range(max(3, args.warmup)):
-        flush.fill_(1)
-        step()
+    def step():
+        for op in ops:
+            op()
+
+    # warm up eagerly, then capture the step (and each op on its own) as CUDA
+    # graphs: the step is launch-bound at its small kernels, and a graph replay
+    # is how the path is meant to be driven
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for _ in range(max(3, args.warmup)):
+            flush.fill_(1)
+            step()
+    stream.wait_stream(side)
     torch.cuda.synchronize()
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step):
+        step()
+    for _ in range(3):
+        flush.fill_(1)
+        g_step.replay()
+    torch.cuda.synchronize()
+    m.moe_check(ws)
 
     K = args.steps
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(K)]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
     sampler = ClockSampler(local) if rank == 0 else None
     if dist is not None:
         dist.barrier()
@@ -356,24 +380,43 @@ def main():
         time.sleep(0.3)
     for i in range(K):
         flush.fill_(1)
-        step(events[i])
+        ev[i][0].record(stream)
+        g_step.replay()
+        ev[i][1].record(stream)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
     m.moe_check(ws)
-
-    seg = [[0.0] * 4 for _ in range(K)]
-    for i in range(K):
-        for s in range(4):
-            seg[i][s] = events[i][s].elapsed_time(events[i][s + 1])  # ms
-    total_ms = sum(sum(r) for r in seg)
-    mean = [sum(seg[i][s] for i in range(K)) / K for s in range(4)]
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
     if dist is not None:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
+
+    # per-kernel breakdown: a probe graph of the same step with event-record
+    # nodes between the kernels, replayed after an L2 flush and read back one
+    # replay at a time
+    n_ops = len(ops)
+    probe_ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ops + 1)]
+    g_probe = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_probe):
+        cap = torch.cuda.current_stream(dev)
+        probe_ev[0].record(cap)
+        for j, op in enumerate(ops):
+            op()
+            probe_ev[j + 1].record(cap)
+    K_ops = max(20, min(400, K // 10))
+    sums = [0.0] * n_ops
+    for i in range(K_ops):
+        flush.fill_(1)
+        g_probe.replay()
+        torch.cuda.synchronize()
+        for j in range(n_ops):
+            sums[j] += probe_ev[j].elapsed_time(probe_ev[j + 1])
+    mean = [v / K_ops for v in sums]
+    del g_probe
 
     # end to end through the public API: pinned host inputs in, result out
     e2e = None
@@ -389,7 +432,7 @@ def main():
                 e0.record(stream)
             x.copy_(x_h, non_blocking=True)
             logits.copy_(lg_h, non_blocking=True)
-            step()
+            g_step.replay()
             out_h.copy_(out, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
@@ -415,9 +458,11 @@ def main():
         gbs = byts[name] / (mean[s] * 1e-3) / 1e9
         kern[name] = {"us": round(us, 2), "bytes": byts[name], "gbs": round(gbs, 1),
                       "frac": round(gbs / peak, 4)}
-    dom = "dispatch" if mean[2] >= mean[3] else "combine"
-    dom_gbs = byts[dom] / (mean[names.index(dom)] * 1e-3) / 1e9
-    dc_ms = mean[2] + mean[3]
+    t_disp = mean[names.index("dispatch")]
+    t_comb = mean[names.index("combine")]
+    dom = "dispatch" if t_disp >= t_comb else "combine"
+    dom_gbs = byts[dom] / (max(t_disp, t_comb) * 1e-3) / 1e9
+    dc_ms = t_disp + t_comb
     dc_gbs = (byts["dispatch"] + byts["combine"]) / (dc_ms * 1e-3) / 1e9
     ms_step = total_ms / K
     line = {
@@ -437,7 +482,7 @@ def main():
                    "k": k, "ranks": w.R, "capacity": w.capacity, "rows": N,
                    "kept_rows": kept_rows, "parallelism": f"replicas x{world}",
                    "l2": "256 MiB write between timed steps, outside the step events",
-                   "step": "route + layout(count, place) + dispatch + combine"},
+                   "step": " + ".join(names) + ", one CUDA graph"},
         "dispatch_combine": {"tokens_per_s": world * T / (dc_ms * 1e-3),
                              "us": round(dc_ms * 1e3, 2), "gbs": round(dc_gbs, 1),
                              "frac": round(dc_gbs / peak, 4),
@@ -447,7 +492,7 @@ def main():
                      "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
                      "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
                      "traffic": ncu_traffic(dom, w.name)},
-        "gpu_launches": 5 * K,
+        "gpu_launches": len(ops) * K,
         "clocks": clocks,
         "e2e": e2e,
     }

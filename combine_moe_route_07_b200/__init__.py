@@ -27,6 +27,7 @@ from . import _binding
 from ._binding import MoeError, MOE_F_FP8, MOE_F_RENORM
 
 __all__ = ["MoeShape", "Workspace", "Layout", "MoeError", "moe_route", "moe_layout",
+           "moe_route_layout",
            "moe_dispatch", "moe_combine", "moe_get_device_error", "moe_check",
            "moe_layout_rows", "moe_workspace_bytes"]
 
@@ -156,6 +157,35 @@ def moe_layout(shape: MoeShape, ids: torch.Tensor, *, ws: Workspace,
         _ptr(out.src_idx, "src_idx", torch.int32, (N,)), ws.ptr, ws.nbytes, _stream(dev))
     _check(st, "moe_layout")
     return out
+
+
+def moe_route_layout(shape: MoeShape, logits: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                     *, ws: Workspace, ids: Optional[torch.Tensor] = None,
+                     gates: Optional[torch.Tensor] = None, out: Optional[Layout] = None):
+    """moe_route then moe_layout in one launch; returns (ids, gates, Layout)."""
+    T, E, k, R = shape.tokens, shape.experts, shape.k, shape.ranks
+    N = shape.rows
+    dev = logits.device
+    i32 = dict(dtype=torch.int32, device=dev)
+    if ids is None:
+        ids = torch.empty((T, k), **i32)
+    if gates is None:
+        gates = torch.empty((T, k), dtype=torch.float32, device=dev)
+    if out is None:
+        out = Layout(torch.empty(E, **i32), torch.empty(E + 1, **i32), torch.empty(R + 1, **i32),
+                     torch.empty(R, **i32), torch.empty((T, k), **i32), torch.empty(N, **i32))
+    st = _binding.lib().moe_route_layout(
+        ctypes.byref(shape.c()), _ptr(logits, "logits", torch.float32, (T, E)),
+        _ptr(bias, "bias", torch.float32, (E,)), _ptr(ids, "ids", torch.int32, (T, k)),
+        _ptr(gates, "gates", torch.float32, (T, k)),
+        _ptr(out.counts, "counts", torch.int32, (E,)),
+        _ptr(out.expert_off, "expert_off", torch.int32, (E + 1,)),
+        _ptr(out.rank_off, "rank_off", torch.int32, (R + 1,)),
+        _ptr(out.rank_counts, "rank_counts", torch.int32, (R,)),
+        _ptr(out.dst_pos, "dst_pos", torch.int32, (T, k)),
+        _ptr(out.src_idx, "src_idx", torch.int32, (N,)), ws.ptr, ws.nbytes, _stream(dev))
+    _check(st, "moe_route_layout")
+    return ids, gates, out
 
 
 def moe_dispatch(shape: MoeShape, x: torch.Tensor, dst_pos: torch.Tensor, *, ws: Workspace,

@@ -153,6 +153,34 @@ moe_status_t moe_layout(const moe_shape_t* shape, const int32_t* ids, int32_t* c
                                       dst_pos, src_idx, kLayoutTimeoutNs));
 }
 
+moe_status_t moe_route_layout(const moe_shape_t* shape, const float* logits, const float* bias,
+                              int32_t* ids, float* gates, int32_t* counts, int32_t* expert_off,
+                              int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
+                              int32_t* src_idx, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!shape_ok(shape)) return MOE_ERR_INVALID_ARG;
+  const int64_t N = rows_of(shape);
+  if (counts == nullptr || expert_off == nullptr || rank_off == nullptr ||
+      rank_counts == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (shape->tokens > 0 && (logits == nullptr || ids == nullptr || gates == nullptr ||
+                            dst_pos == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (N > 0 && src_idx == nullptr) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {logits, bias, ids, gates, counts, expert_off, rank_off, rank_counts,
+                        dst_pos, src_idx};
+  for (const void* p : ptrs)
+    if (!aligned(p, 4)) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = ws_ok(shape, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  WsHeader* hdr = static_cast<WsHeader*>(ws);
+  uint32_t* table = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + kHeaderBytes);
+  return from_cuda(moe::launch_route_layout(
+      env_of(stream), logits, bias, (shape->flags & MOE_F_RENORM) ? 1 : 0, ids, gates,
+      shape->tokens, shape->experts, shape->k, shape->ranks, shape->capacity, shape->align, N,
+      table, hdr, counts, expert_off, rank_off, rank_counts, dst_pos, src_idx,
+      kLayoutTimeoutNs));
+}
+
 moe_status_t moe_dispatch(const moe_shape_t* shape, const void* x, const int32_t* dst_pos,
                           void* out, float* scales, void* ws, size_t ws_bytes,
                           moe_stream_t stream) {

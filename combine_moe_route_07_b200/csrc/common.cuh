@@ -13,10 +13,12 @@ constexpr unsigned kFull = 0xffffffffu;
 
 // Workspace header (first 256 bytes of every workspace).
 struct WsHeader {
-  int32_t err;      // first device-side error code (moe_status_t), 0 = none
-  int32_t detail;   // index that caused it
-  uint32_t ticket;  // layout: next virtual block id; reset by the last block
-  uint32_t pad[61];
+  int32_t err;            // first device-side error code (moe_status_t), 0 = none
+  int32_t detail;         // index that caused it
+  uint32_t looked;        // layout: tiles whose lookback is done
+  uint32_t totals_ready;  // layout: expert offsets are published
+  uint32_t finished;      // layout: tiles that are done; the last one resets the three
+  uint32_t pad[59];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 
@@ -39,6 +41,16 @@ __device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
 __device__ __forceinline__ void st_relaxed(uint32_t* p, uint32_t v) {
   asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// L2-coherent 32-bit load (bypasses L1), for data another CTA published.
+__device__ __forceinline__ int32_t ld_cg(const int32_t* p) { return __ldcg(p); }
 
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;

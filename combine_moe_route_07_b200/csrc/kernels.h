@@ -14,7 +14,8 @@ struct LaunchEnv {
   int num_sms;
 };
 
-// Tokens per layout tile (one CTA of each layout kernel per tile).
+// Tokens per layout tile (one CTA per tile); the launch doubles it while the
+// tiles outnumber the CTAs that fit on the GPU at once.
 constexpr int kLayoutTileTokens = 128;
 
 cudaError_t launch_route(const LaunchEnv& env, const float* logits, const float* bias, int T,
@@ -25,6 +26,13 @@ cudaError_t launch_layout(const LaunchEnv& env, const int32_t* ids, int T, int E
                           int32_t* counts, int32_t* expert_off, int32_t* rank_off,
                           int32_t* rank_counts, int32_t* dst_pos, int32_t* src_idx,
                           uint64_t timeout_ns);
+
+cudaError_t launch_route_layout(const LaunchEnv& env, const float* logits, const float* bias,
+                                int renorm, int32_t* ids, float* gates, int T, int E, int k,
+                                int R, int capacity, int align, int64_t N, uint32_t* table,
+                                WsHeader* hdr, int32_t* counts, int32_t* expert_off,
+                                int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
+                                int32_t* src_idx, uint64_t timeout_ns);
 
 cudaError_t launch_dispatch_bf16(const LaunchEnv& env, const void* x, const int32_t* dst_pos,
                                  int T, int H, int k, int64_t N, void* out, WsHeader* hdr);

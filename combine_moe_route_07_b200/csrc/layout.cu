@@ -1,4 +1,5 @@
-// layout.cu -- steps 2 and 3: per-expert count histogram and the layout scan.
+// layout.cu -- steps 2 and 3: per-expert count histogram and the layout scan
+// (optionally fused with step 1, the router).
 //
 // "GPU MoE all-to-all" (aicassindra), section "Two collectives per layer":
 // per-destination counts precede the payload; section "Bucketing": sort rows
@@ -9,29 +10,29 @@
 // each destination's rows form one contiguous band (experts are numbered
 // rank-major, so rank slices are unions of consecutive expert segments).
 //
-// Two kernels over tiles of kLayoutTileTokens tokens:
+// One cooperative kernel, one CTA per tile of TT tokens (all CTAs resident at
+// once, so CTAs may wait on one another; every wait is bounded):
 //
-//  count  one CTA per tile, virtual tile id from an atomic ticket (so every
-//         tile a CTA waits on belongs to a CTA that is already running).
-//         Shared-memory histogram of the tile's expert ids, then a
-//         decoupled-lookback scan across tiles, per expert: publish the
-//         tile's aggregate, walk back over predecessors until an inclusive
-//         prefix is found, publish the inclusive prefix.  Flag and value
-//         share one 32-bit word (flag in bits 30-31), so a relaxed store is
-//         enough.  The CTA holding the last tile sees the totals and writes
-//         counts, expert/rank offsets and per-rank kept counts.
-//  place  one CTA per tile again.  Warps own contiguous runs of the tile's
-//         assignments; per-warp histograms (__match_any_sync, leader adds)
-//         and a scan over warps give each assignment its token-order rank
-//         inside its expert with no atomics, so the result never depends on
-//         scheduling.  Writes dst_pos / src_idx, marks padding rows -1 and
-//         leaves the lookback table and ticket zeroed for the next call.
-//
-// Every wait is bounded: after `timeout_ns` it records
-// MOE_ERR_DEVICE_TIMEOUT, publishes a placeholder so successors stop
-// waiting, and returns.
+//  1. (fused variant) route the tile's tokens, one warp per token.
+//  2. Per-warp histograms of the tile's expert ids over contiguous runs of
+//     assignments (__match_any_sync; the run leader adds), summed into the
+//     tile histogram.  No atomics, so no result depends on scheduling.
+//  3. Decoupled lookback across tiles, per expert, in an expert-major table:
+//     publish the tile's aggregate, read a window of 32 predecessors at once,
+//     add back to the nearest inclusive prefix, publish the inclusive prefix.
+//     Flag and value share one 32-bit word (flag in bits 30-31).
+//  4. The CTA of the last tile holds the totals: counts, expert offsets
+//     (segments rounded to `align`, or C rows each), rank offsets and kept
+//     rows per rank; it publishes them and raises a ready flag.
+//  5. Every CTA places its assignments: token-order rank inside the expert =
+//     tile prefix + warp prefix + lane rank within the run; capacity mode
+//     keeps ranks < C.  Writes dst_pos / src_idx and marks its share of the
+//     padding rows -1.
+//  6. Once every lookback is done, each CTA clears its table column; the last
+//     CTA to finish resets the counters, leaving the workspace ready.
 #include "common.cuh"
 #include "kernels.h"
+#include "route_core.cuh"
 
 namespace moe {
 
@@ -39,27 +40,88 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+constexpr int kWindow = 32;
+constexpr int kUnroll = 4;
 constexpr uint32_t kFlagAgg = 1u << 30;
 constexpr uint32_t kFlagIncl = 2u << 30;
 constexpr uint32_t kValMask = (1u << 30) - 1u;
 constexpr unsigned kMaxSpins = 1u << 26;
 
-__device__ uint32_t wait_published(const uint32_t* p, WsHeader* hdr, uint64_t timeout_ns,
-                                   int who) {
-  uint32_t w = ld_relaxed(p);
-  if (w & ~kValMask) return w;
+struct LayoutParams {
+  const int32_t* ids;  // [T,k]: input, or written by step 1 in the fused kernel
+  int32_t* ids_out;    // fused: where step 1 writes the ids (same buffer)
+  const float* logits;
+  const float* bias;
+  float* gates;
+  int renorm;
+  int T, k, E, R, capacity, align, B, TT;
+  int64_t N;
+  uint32_t* table;  // [E][B] lookback words
+  WsHeader* hdr;
+  int32_t* counts;
+  int32_t* expert_off;
+  int32_t* rank_off;
+  int32_t* rank_counts;
+  int32_t* dst_pos;
+  int32_t* src_idx;
+  uint64_t timeout_ns;
+};
+
+// Wait until the word at p carries a flag; after the time limit record
+// MOE_ERR_DEVICE_TIMEOUT and return a placeholder inclusive 0.
+__device__ __noinline__ uint32_t wait_word(const uint32_t* p, WsHeader* hdr, uint64_t timeout_ns,
+                                           int who) {
   const uint64_t t0 = global_ns();
-  for (unsigned it = 1; it < kMaxSpins; ++it) {
-    __nanosleep(64);
-    w = ld_relaxed(p);
+  for (unsigned it = 0; it < kMaxSpins; ++it) {
+    const uint32_t w = ld_relaxed(p);
     if (w & ~kValMask) return w;
-    if ((it & 15u) == 0u) {
+    if ((it & 15u) == 15u) {
       if (error_seen(hdr) == MOE_ERR_DEVICE_TIMEOUT) return kFlagIncl;
       if (global_ns() - t0 > timeout_ns) break;
     }
+    __nanosleep(64);
   }
   report(hdr, MOE_ERR_DEVICE_TIMEOUT, who);
   return kFlagIncl;
+}
+
+// Wait until *p >= target; false (and MOE_ERR_DEVICE_TIMEOUT) after the limit.
+__device__ __noinline__ bool wait_count(const uint32_t* p, uint32_t target, WsHeader* hdr,
+                                        uint64_t timeout_ns, int who) {
+  const uint64_t t0 = global_ns();
+  for (unsigned it = 0; it < kMaxSpins; ++it) {
+    if (ld_acquire(p) >= target) return true;
+    if ((it & 15u) == 15u) {
+      if (error_seen(hdr) == MOE_ERR_DEVICE_TIMEOUT) return false;
+      if (global_ns() - t0 > timeout_ns) break;
+    }
+    __nanosleep(128);
+  }
+  report(hdr, MOE_ERR_DEVICE_TIMEOUT, who);
+  return false;
+}
+
+// Exclusive prefix of tile vb for one expert: sum the predecessors' words from
+// the nearest back to the first inclusive one, 32 loads in flight at a time.
+__device__ uint32_t lookback(const uint32_t* col, int vb, WsHeader* hdr, uint64_t timeout_ns) {
+  uint32_t excl = 0;
+  for (int hi = vb - 1; hi >= 0; hi -= kWindow) {
+    uint32_t w[kWindow];
+#pragma unroll
+    for (int i = 0; i < kWindow; ++i) w[i] = (hi - i >= 0) ? ld_relaxed(col + hi - i) : 0u;
+    bool done = false;
+#pragma unroll
+    for (int i = 0; i < kWindow; ++i) {
+      if (!done && hi - i >= 0) {
+        uint32_t v = w[i];
+        if ((v & ~kValMask) == 0u) v = wait_word(col + hi - i, hdr, timeout_ns, vb);
+        excl += v & kValMask;
+        done = (v & ~kValMask) == kFlagIncl;
+      }
+    }
+    if (done) break;
+  }
+  return excl & kValMask;
 }
 
 // Exclusive scan of v[0..n) in shared memory by the whole CTA (n <= 4 *
@@ -101,211 +163,310 @@ __device__ int block_exclusive_scan(int32_t* v, int n, int32_t* warp_tot) {
   return total;
 }
 
-__global__ void __launch_bounds__(kThreads)
-    layout_count_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int R, int capacity,
-                        int align, int B, uint32_t* __restrict__ status, WsHeader* hdr,
-                        int32_t* __restrict__ counts, int32_t* __restrict__ expert_off,
-                        int32_t* __restrict__ rank_off, int32_t* __restrict__ rank_counts,
-                        uint64_t timeout_ns) {
+template <int NK, bool ROUTE>
+__global__ void __launch_bounds__(kThreads) layout_kernel(const LayoutParams P) {
   extern __shared__ int32_t smem[];
-  int32_t* hist = smem;     // [E] this tile's histogram, later the segment scan
-  int32_t* tot = smem + E;  // [E] inclusive prefix through this tile
-  __shared__ uint32_t s_vb;
-  __shared__ int32_t s_wtot[kWarps];
-
-  if (threadIdx.x == 0) s_vb = atomicAdd(&hdr->ticket, 1u);
-  for (int e = threadIdx.x; e < E; e += kThreads) hist[e] = 0;
-  __syncthreads();
-  const int vb = (int)s_vb;
-  if (vb >= B) {  // only with a workspace that was not left zeroed
-    if (threadIdx.x == 0) report(hdr, MOE_ERR_WORKSPACE, vb);
-    return;
-  }
-
-  const int64_t i0 = (int64_t)vb * kLayoutTileTokens * k;
-  const int64_t i1 = (int64_t)min(T, (vb + 1) * kLayoutTileTokens) * k;
-  for (int64_t i = i0 + threadIdx.x; i < i1; i += kThreads) {
-    const int e = __ldg(ids + i);
-    if ((unsigned)e < (unsigned)E)
-      atomicAdd(&hist[e], 1);
-    else
-      report(hdr, MOE_ERR_DEVICE_RANGE, (int)i);
-  }
-  __syncthreads();
-
-  uint32_t* mine = status + (size_t)vb * E;
-  const uint32_t flag0 = (vb == 0) ? kFlagIncl : kFlagAgg;
-  for (int e = threadIdx.x; e < E; e += kThreads) st_relaxed(mine + e, flag0 | (uint32_t)hist[e]);
-
-  for (int e = threadIdx.x; e < E; e += kThreads) {
-    uint32_t excl = 0;
-    for (int p = vb - 1; p >= 0; --p) {
-      const uint32_t w = wait_published(status + (size_t)p * E + e, hdr, timeout_ns, vb);
-      excl += w & kValMask;
-      if ((w & ~kValMask) == kFlagIncl) break;
-    }
-    const uint32_t incl = (excl + (uint32_t)hist[e]) & kValMask;
-    if (vb > 0) st_relaxed(mine + e, kFlagIncl | incl);
-    tot[e] = (int32_t)incl;
-  }
-
-  if (vb != B - 1) return;
-  // The last tile's inclusive prefixes are the totals.
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += kThreads) {
-    const int c = tot[e];
-    counts[e] = c;
-    hist[e] = capacity > 0 ? capacity : ((c + align - 1) / align) * align;
-    tot[e] = (capacity > 0 && c > capacity) ? capacity : c;  // kept
-  }
-  __syncthreads();
-  const int used = block_exclusive_scan(hist, E, s_wtot);
-  const int kept_total = block_exclusive_scan(tot, E, s_wtot);
-  for (int e = threadIdx.x; e < E; e += kThreads) expert_off[e] = hist[e];
-  const int Er = E / R;
-  for (int r = threadIdx.x; r < R; r += kThreads) {
-    rank_off[r] = hist[r * Er];
-    const int hi = (r + 1 < R) ? tot[(r + 1) * Er] : kept_total;
-    rank_counts[r] = hi - tot[r * Er];
-  }
-  if (threadIdx.x == 0) {
-    expert_off[E] = used;
-    rank_off[R] = used;
-  }
-}
-
-__global__ void __launch_bounds__(kThreads)
-    layout_place_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int capacity, int B,
-                        int64_t N, int fill, uint32_t* __restrict__ status, WsHeader* hdr,
-                        const int32_t* __restrict__ counts, const int32_t* __restrict__ expert_off,
-                        int32_t* __restrict__ dst_pos, int32_t* __restrict__ src_idx) {
-  extern __shared__ int32_t smem[];
-  int32_t* wh = smem;                // [kWarps][E] per-warp counters
-  int32_t* off = smem + kWarps * E;  // [E+1]  (padding fill)
+  const int E = P.E, k = P.k, C = P.capacity;
+  int32_t* wh = smem;                // [kWarps][E] per-warp counts, then bases
+  int32_t* tile = wh + kWarps * E;   // [E] tile histogram, then inclusive prefix
+  int32_t* off = tile + E;           // [E+1] expert offsets
   int32_t* kept = off + E + 1;       // [E]
+  __shared__ int32_t s_wtot[kWarps];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.x;
+  const int vb = blockIdx.x;
+  const int t0 = min(P.T, vb * P.TT);
+  const int t1 = min(P.T, t0 + P.TT);
 
-  if (b == 0 && threadIdx.x == 0) hdr->ticket = 0u;  // the count pass is over
+  if constexpr (ROUTE) {
+    float b[NK];
+    load_bias<NK>(P.bias, E, lane, b);
+    for (int t = t0 + w; t < t1; t += kWarps) {
+      int e;
+      float g;
+      bool nan_key;
+      route_token<NK>(P.logits + (size_t)t * E, b, E, k, P.renorm, lane, e, g, nan_key);
+      if (nan_key && lane == 0) report(P.hdr, MOE_ERR_DEVICE_NAN, t);
+      if (lane < k) {
+        P.ids_out[(size_t)t * k + lane] = e;
+        P.gates[(size_t)t * k + lane] = g;
+      }
+    }
+  }
   for (int i = threadIdx.x; i < kWarps * E; i += kThreads) wh[i] = 0;
-  __syncthreads();
+  __syncthreads();  // (fused) the tile's ids are written before anyone reads them
 
-  const int64_t i0 = (int64_t)b * kLayoutTileTokens * k;
-  const int64_t i1 = (int64_t)min(T, (b + 1) * kLayoutTileTokens) * k;
-  const int64_t n = i1 - i0;
-  const int64_t chunk = (((n + kWarps - 1) / kWarps) + 31) / 32 * 32;
+  // this warp's contiguous run of the tile's assignments
+  const int64_t i0 = (int64_t)t0 * k, i1 = (int64_t)t1 * k;
+  const int64_t chunk = (((i1 - i0) + kWarps - 1) / kWarps + 31) / 32 * 32;
   const int64_t s0 = min(i1, i0 + (int64_t)w * chunk);
   const int64_t s1 = min(i1, s0 + chunk);
   int32_t* my = wh + w * E;
 
-  // pass 1: per-warp histogram of this warp's run
-  for (int64_t base = s0; base < s1; base += 32) {
-    const int64_t i = base + lane;
-    const int e = (i < s1) ? __ldg(ids + i) : -1;
-    const bool ok = (i < s1) && (unsigned)e < (unsigned)E;
-    const unsigned active = __ballot_sync(kFull, ok);
-    if (ok) {
-      const unsigned peers = __match_any_sync(active, e);
-      if (lane == __ffs(peers) - 1) my[e] += __popc(peers);
+  // pass 1: per-warp histogram
+  for (int64_t base = s0; base < s1; base += 32 * kUnroll) {
+    int ev[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t i = base + 32 * u + lane;
+      ev[u] = (i < s1) ? P.ids[i] : -1;
     }
-    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t i = base + 32 * u + lane;
+      if (base + 32 * u < s1) {
+        const bool ok = (i < s1) && (unsigned)ev[u] < (unsigned)E;
+        if (i < s1 && !ok) report(P.hdr, MOE_ERR_DEVICE_RANGE, (int)i);
+        const unsigned active = __ballot_sync(kFull, ok);
+        if (ok) {
+          const unsigned peers = __match_any_sync(active, ev[u]);
+          if (lane == __ffs(peers) - 1) my[ev[u]] += __popc(peers);
+        }
+        __syncwarp();
+      }
+    }
   }
   __syncthreads();
 
-  // first row (dropless) or first token-order rank (capacity) of each warp's
-  // share of each expert
+  // tile histogram; publish the aggregate (tile 0: its inclusive prefix)
   for (int e = threadIdx.x; e < E; e += kThreads) {
     int h = 0;
     for (int q = 0; q < kWarps; ++q) h += wh[q * E + e];
-    const int incl = (int)(status[(size_t)b * E + e] & kValMask);
-    int run = (capacity > 0 ? 0 : expert_off[e]) + (incl - h);
+    tile[e] = h;
+    st_relaxed(P.table + (size_t)e * P.B + vb, (vb == 0 ? kFlagIncl : kFlagAgg) | (uint32_t)h);
+  }
+  // lookback; then each warp's first token-order rank in each expert
+  for (int e = threadIdx.x; e < E; e += kThreads) {
+    const uint32_t ex = (vb > 0) ? lookback(P.table + (size_t)e * P.B, vb, P.hdr, P.timeout_ns)
+                                 : 0u;
+    if (vb > 0)
+      st_relaxed(P.table + (size_t)e * P.B + vb, kFlagIncl | ((ex + (uint32_t)tile[e]) & kValMask));
+    int run = (int)ex;
     for (int q = 0; q < kWarps; ++q) {
       const int c = wh[q * E + e];
       wh[q * E + e] = run;
       run += c;
     }
-    status[(size_t)b * E + e] = 0u;
+    tile[e] = run;
   }
   __syncthreads();
-
-  // pass 2: rank inside the warp's step, in lane (= token) order
-  for (int64_t base = s0; base < s1; base += 32) {
-    const int64_t i = base + lane;
-    const int e = (i < s1) ? __ldg(ids + i) : -1;
-    const bool ok = (i < s1) && (unsigned)e < (unsigned)E;
-    const unsigned active = __ballot_sync(kFull, ok);
-    int v = 0, cnt = 0;
-    bool lead = false;
-    if (ok) {
-      const unsigned peers = __match_any_sync(active, e);
-      v = my[e] + __popc(peers & lanemask_lt());
-      lead = (lane == __ffs(peers) - 1);
-      cnt = __popc(peers);
-    }
-    __syncwarp();
-    if (lead) my[e] = v + cnt;
-    __syncwarp();
-    if (i < s1) {
-      int dst = -1;
-      if (ok) dst = (capacity > 0) ? (v < capacity ? e * capacity + v : -1) : v;
-      // Positions are in range by construction; the check only matters after
-      // a count pass that gave up (its prefixes are placeholders).
-      if (dst >= N || (ok && v < 0)) {
-        report(hdr, MOE_ERR_DEVICE_RANGE, dst);
-        dst = -1;
-      }
-      dst_pos[i] = dst;
-      if (dst >= 0) src_idx[dst] = (int32_t)i;
-    }
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(&P.hdr->looked, 1u);
   }
 
-  if (!fill) return;
-  // rows that hold no assignment: alignment padding, unused capacity slots
-  for (int e = threadIdx.x; e <= E; e += kThreads) off[e] = expert_off[e];
-  for (int e = threadIdx.x; e < E; e += kThreads) {
-    const int c = counts[e];
-    kept[e] = (capacity > 0 && c > capacity) ? capacity : c;
+  // the last tile's inclusive prefixes are the totals
+  if (vb == P.B - 1) {
+    for (int e = threadIdx.x; e < E; e += kThreads) {
+      const int c = tile[e];
+      P.counts[e] = c;
+      off[e] = C > 0 ? C : ((c + P.align - 1) / P.align) * P.align;
+      kept[e] = (C > 0 && c > C) ? C : c;
+    }
+    __syncthreads();
+    const int used = block_exclusive_scan(off, E, s_wtot);
+    const int kept_total = block_exclusive_scan(kept, E, s_wtot);
+    const int Er = E / P.R;
+    for (int e = threadIdx.x; e < E; e += kThreads) P.expert_off[e] = off[e];
+    for (int r = threadIdx.x; r < P.R; r += kThreads) {
+      P.rank_off[r] = off[r * Er];
+      const int hi = (r + 1 < P.R) ? kept[(r + 1) * Er] : kept_total;
+      P.rank_counts[r] = hi - kept[r * Er];
+    }
+    if (threadIdx.x == 0) {
+      P.expert_off[E] = used;
+      P.rank_off[P.R] = used;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      st_release(&P.hdr->totals_ready, 1u);
+    }
   }
+  if (threadIdx.x == 0) wait_count(&P.hdr->totals_ready, 1u, P.hdr, P.timeout_ns, vb);
   __syncthreads();
-  const int64_t per = (N + B - 1) / B;
-  const int64_t r0 = (int64_t)b * per;
-  const int64_t r1 = min(N, r0 + per);
-  for (int64_t p = r0 + threadIdx.x; p < r1; p += kThreads) {
-    bool pad = true;
-    if (p < off[E]) {
-      int lo = 0, hi = E - 1;  // last e with off[e] <= p
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (off[mid] <= p)
-          lo = mid;
-        else
-          hi = mid - 1;
-      }
-      pad = (p - off[lo]) >= kept[lo];
+  const bool fill = (C > 0 || P.align > 1);
+  for (int e = threadIdx.x; e <= E; e += kThreads) off[e] = ld_cg(P.expert_off + e);
+  if (fill)
+    for (int e = threadIdx.x; e < E; e += kThreads) {
+      const int c = ld_cg(P.counts + e);
+      kept[e] = (C > 0 && c > C) ? C : c;
     }
-    if (pad) src_idx[p] = -1;
+  __syncthreads();
+
+  // pass 2: place each assignment at its token-order rank
+  for (int64_t base = s0; base < s1; base += 32 * kUnroll) {
+    int ev[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t i = base + 32 * u + lane;
+      ev[u] = (i < s1) ? P.ids[i] : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t i = base + 32 * u + lane;
+      if (base + 32 * u < s1) {
+        const int e = ev[u];
+        const bool ok = (i < s1) && (unsigned)e < (unsigned)E;
+        const unsigned active = __ballot_sync(kFull, ok);
+        int v = 0, cnt = 0;
+        bool lead = false;
+        if (ok) {
+          const unsigned peers = __match_any_sync(active, e);
+          v = my[e] + __popc(peers & lanemask_lt());
+          lead = (lane == __ffs(peers) - 1);
+          cnt = __popc(peers);
+        }
+        __syncwarp();
+        if (lead) my[e] = v + cnt;
+        __syncwarp();
+        if (i < s1) {
+          int64_t dst = -1;
+          if (ok) dst = (C > 0) ? (v < C ? (int64_t)e * C + v : -1) : (int64_t)off[e] + v;
+          // in range by construction; checked because a lookback that gave up
+          // leaves placeholder prefixes
+          if (dst >= P.N || (ok && v < 0)) {
+            report(P.hdr, MOE_ERR_DEVICE_RANGE, (int)dst);
+            dst = -1;
+          }
+          P.dst_pos[i] = (int32_t)dst;
+          if (dst >= 0) P.src_idx[dst] = (int32_t)i;
+        }
+      }
+    }
   }
+
+  // rows that hold no assignment (alignment padding, unused capacity slots)
+  if (fill) {
+    const int64_t per = (P.N + P.B - 1) / P.B;
+    const int64_t r0 = (int64_t)vb * per;
+    const int64_t r1 = min(P.N, r0 + per);
+    for (int64_t p = r0 + threadIdx.x; p < r1; p += kThreads) {
+      bool pad = true;
+      if (p < off[E]) {
+        int lo = 0, hi = E - 1;  // last e with off[e] <= p
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (off[mid] <= p)
+            lo = mid;
+          else
+            hi = mid - 1;
+        }
+        pad = (p - off[lo]) >= kept[lo];
+      }
+      if (pad) P.src_idx[p] = -1;
+    }
+  }
+
+  // once no lookback reads the table any more, clear this tile's column
+  if (threadIdx.x == 0) wait_count(&P.hdr->looked, (uint32_t)P.B, P.hdr, P.timeout_ns, vb);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kThreads) P.table[(size_t)e * P.B + vb] = 0u;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&P.hdr->finished, 1u) == (uint32_t)P.B - 1u) {
+      P.hdr->looked = 0u;
+      P.hdr->totals_ready = 0u;
+      P.hdr->finished = 0u;
+    }
+  }
+}
+
+template <int NK, bool ROUTE>
+cudaError_t launch_fused(const LaunchEnv& env, LayoutParams P) {
+  auto kern = layout_kernel<NK, ROUTE>;
+  const size_t smem = (11 * (size_t)P.E + 1) * sizeof(int32_t);
+  int per_sm = 0;
+  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+  if (err != cudaSuccess) return err;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const int64_t max_blocks = (int64_t)per_sm * env.num_sms;
+  // tiles of 128 tokens, doubled until every tile's CTA can be resident at once
+  int64_t TT = kLayoutTileTokens;
+  int64_t B = P.T > 0 ? (P.T + TT - 1) / TT : 1;
+  while (B > max_blocks) {
+    TT *= 2;
+    B = (P.T + TT - 1) / TT;
+  }
+  P.TT = (int)TT;
+  P.B = (int)B;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)B);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = env.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, P);
 }
 
 }  // namespace
 
 cudaError_t launch_layout(const LaunchEnv& env, const int32_t* ids, int T, int E, int k, int R,
-                          int capacity, int align, int64_t N, uint32_t* status, WsHeader* hdr,
+                          int capacity, int align, int64_t N, uint32_t* table, WsHeader* hdr,
                           int32_t* counts, int32_t* expert_off, int32_t* rank_off,
                           int32_t* rank_counts, int32_t* dst_pos, int32_t* src_idx,
                           uint64_t timeout_ns) {
-  const int B = T > 0 ? (T + kLayoutTileTokens - 1) / kLayoutTileTokens : 1;
-  const size_t smem_count = (size_t)2 * E * sizeof(int32_t);
-  layout_count_kernel<<<B, kThreads, smem_count, env.stream>>>(
-      ids, T, k, E, R, capacity, align, B, status, hdr, counts, expert_off, rank_off, rank_counts,
-      timeout_ns);
-  cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
-  const int fill = (capacity > 0 || align > 1) ? 1 : 0;
-  const size_t smem_place = ((size_t)kWarps * E + 2 * (size_t)E + 1) * sizeof(int32_t);
-  layout_place_kernel<<<B, kThreads, smem_place, env.stream>>>(
-      ids, T, k, E, capacity, B, N, fill, status, hdr, counts, expert_off, dst_pos, src_idx);
-  return cudaGetLastError();
+  LayoutParams P{};
+  P.ids = ids;
+  P.T = T;
+  P.k = k;
+  P.E = E;
+  P.R = R;
+  P.capacity = capacity;
+  P.align = align;
+  P.N = N;
+  P.table = table;
+  P.hdr = hdr;
+  P.counts = counts;
+  P.expert_off = expert_off;
+  P.rank_off = rank_off;
+  P.rank_counts = rank_counts;
+  P.dst_pos = dst_pos;
+  P.src_idx = src_idx;
+  P.timeout_ns = timeout_ns;
+  return launch_fused<1, false>(env, P);
+}
+
+cudaError_t launch_route_layout(const LaunchEnv& env, const float* logits, const float* bias,
+                                int renorm, int32_t* ids, float* gates, int T, int E, int k,
+                                int R, int capacity, int align, int64_t N, uint32_t* table,
+                                WsHeader* hdr, int32_t* counts, int32_t* expert_off,
+                                int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
+                                int32_t* src_idx, uint64_t timeout_ns) {
+  LayoutParams P{};
+  P.ids = ids;
+  P.ids_out = ids;
+  P.logits = logits;
+  P.bias = bias;
+  P.gates = gates;
+  P.renorm = renorm;
+  P.T = T;
+  P.k = k;
+  P.E = E;
+  P.R = R;
+  P.capacity = capacity;
+  P.align = align;
+  P.N = N;
+  P.table = table;
+  P.hdr = hdr;
+  P.counts = counts;
+  P.expert_off = expert_off;
+  P.rank_off = rank_off;
+  P.rank_counts = rank_counts;
+  P.dst_pos = dst_pos;
+  P.src_idx = src_idx;
+  P.timeout_ns = timeout_ns;
+  const int nk = (E + 31) / 32;
+  if (nk <= 1) return launch_fused<1, true>(env, P);
+  if (nk <= 2) return launch_fused<2, true>(env, P);
+  if (nk <= 4) return launch_fused<4, true>(env, P);
+  if (nk <= 8) return launch_fused<8, true>(env, P);
+  if (nk <= 16) return launch_fused<16, true>(env, P);
+  return launch_fused<32, true>(env, P);
 }
 
 }  // namespace moe

@@ -91,8 +91,8 @@ typedef struct {
  * Returns -1 for an invalid shape. */
 int64_t moe_layout_rows(const moe_shape_t* shape);
 
-/* Bytes of device workspace the calls need for `shape` (error word, block
- * ticket and the layout's per-block prefix table).  0 for an invalid shape.
+/* Bytes of device workspace the calls need for `shape` (error word, the
+ * layout's counters and its per-tile prefix table).  0 for an invalid shape.
  * A workspace sized for one shape serves any shape whose requirement is not
  * larger. */
 size_t moe_workspace_bytes(const moe_shape_t* shape);
@@ -135,6 +135,15 @@ moe_status_t moe_layout(const moe_shape_t* shape, const int32_t* ids, int32_t* c
                         int32_t* expert_off, int32_t* rank_off, int32_t* rank_counts,
                         int32_t* dst_pos, int32_t* src_idx, void* ws, size_t ws_bytes,
                         moe_stream_t stream);
+
+/* Steps 1-3 in one launch: moe_route followed by moe_layout, fused so the
+ * ids never leave the CTA that routed them before they are counted.  Same
+ * arguments (the union of both calls), same results bit for bit, same error
+ * behaviour. */
+moe_status_t moe_route_layout(const moe_shape_t* shape, const float* logits, const float* bias,
+                              int32_t* ids, float* gates, int32_t* counts, int32_t* expert_off,
+                              int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
+                              int32_t* src_idx, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Step 4 -- dispatch ("GPU MoE all-to-all", sections "Bucketing" and
  * "Latency-bound at decode, bandwidth-bound at prefill").

@@ -66,24 +66,30 @@ def standin_oracle(w: Workload, disp, L):
 
 # ------------------------------------------------------------ the paths ----
 
-def run_gpu(w: Workload, inp, ids=None, gates=None):
+def run_gpu(w: Workload, inp, ids=None, gates=None, fused=False):
     """Run route (unless ids/gates are given), layout, dispatch, stand-in and
-    combine on cuda:0.  Returns a dict of CUDA tensors and the workspace."""
+    combine on cuda:0 (fused: route and layout in one moe_route_layout call).
+    Returns a dict of CUDA tensors and the workspace."""
     import combine_moe_route_07_b200 as m
     dev = torch.device("cuda:0")
     shape = shape_of(w)
     ws = m.Workspace(shape, dev)
     x = inp.x.to(dev)
     res = {"ws": ws, "x": x}
-    if ids is None:
+    if fused:
+        logits = inp.logits.to(dev)
+        bias = None if inp.bias is None else inp.bias.to(dev)
+        ids, gates, lay = m.moe_route_layout(shape, logits, bias, ws=ws)
+    elif ids is None:
         logits = inp.logits.to(dev)
         bias = None if inp.bias is None else inp.bias.to(dev)
         ids, gates = m.moe_route(shape, logits, bias, ws=ws)
+        lay = m.moe_layout(shape, ids, ws=ws)
     else:
         ids = torch.from_numpy(np.ascontiguousarray(ids)).to(dev)
         gates = torch.from_numpy(np.ascontiguousarray(gates)).to(dev)
+        lay = m.moe_layout(shape, ids, ws=ws)
     res["ids"], res["gates"] = ids, gates
-    lay = m.moe_layout(shape, ids, ws=ws)
     res["layout"] = lay
     disp = m.moe_dispatch(shape, x, lay.dst_pos, ws=ws)
     res["dispatch"] = disp

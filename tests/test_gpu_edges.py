@@ -16,11 +16,11 @@ pytestmark = pytest.mark.gpu
 LAYOUT_KEYS = ("counts", "expert_off", "rank_off", "rank_counts", "dst_pos", "src_idx")
 
 
-def _check_all(w, inp=None):
+def _check_all(w, inp=None, fused=False):
     import combine_moe_route_07_b200 as m
     inp = inp or make_inputs(w)
     o = run_oracle(w, inp)
-    g = run_gpu(w, inp)
+    g = run_gpu(w, inp, fused=fused)
     assert m.moe_get_device_error(g["ws"]) == (0, 0)
     assert np.array_equal(to_np(g["ids"]), o["ids"])
     assert_gates_close(to_np(g["gates"]), o["gates"])
@@ -60,12 +60,15 @@ CASES = [
     Workload("scale_expert_capacity", T=512, H=64, E=16, R=4, k=2, expert="scale",
              capacity_factor=0.8),
     Workload("many_tiles", T=20000, H=16, E=64, R=8, k=6),
+    # more 128-token tiles than CTAs that fit at once: the launch widens tiles
+    Workload("wide_tiles", T=120000, H=8, E=1024, R=8, k=2),
 ]
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
 @pytest.mark.parametrize("w", CASES, ids=[c.name for c in CASES])
-def test_edge_case_parity(w):
-    _check_all(w)
+def test_edge_case_parity(w, fused):
+    _check_all(w, fused=fused)
 
 
 def test_empty_batch():
@@ -98,9 +101,10 @@ def test_all_tokens_on_the_same_experts():
     bias = torch.zeros(16)
     bias[5], bias[2], bias[7] = 300.0, 200.0, 100.0
     inp.bias = bias
-    _check_all(w, inp)
-    wc = w.with_(name="same_experts_capacity", capacity_factor=0.25)
-    _check_all(wc, inp)
+    for fused in (False, True):
+        _check_all(w, inp, fused)
+        wc = w.with_(name="same_experts_capacity", capacity_factor=0.25)
+        _check_all(wc, inp, fused)
 
 
 def test_bad_ids_set_the_device_error_and_are_dropped():

@@ -31,12 +31,13 @@ def _compare_layout(g_lay, L, what):
         assert np.array_equal(got, L[key]), f"{what}: layout.{key} differs"
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
 @pytest.mark.parametrize("name", SMALL)
-def test_full_path_small_configs(name):
+def test_full_path_small_configs(name, fused):
     w = WORKLOADS[name]
     inp = inputs_for(w)
     o = run_oracle(w, inp)
-    g = run_gpu(w, inp)
+    g = run_gpu(w, inp, fused=fused)
     import combine_moe_route_07_b200 as m
     assert m.moe_get_device_error(g["ws"]) == (0, 0)
     assert np.array_equal(to_np(g["ids"]), o["ids"])
@@ -72,13 +73,14 @@ def test_each_kernel_on_oracle_inputs(name):
 
 
 @pytest.mark.slow
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
 @pytest.mark.parametrize("name", BIG)
-def test_full_size_route_layout_exact_and_sampled_payload(name):
+def test_full_size_route_layout_exact_and_sampled_payload(name, fused):
     import combine_moe_route_07_b200 as m
     w = WORKLOADS[name]
     inp = inputs_for(w)
     o = run_oracle(w, inp, through="layout")
-    g = run_gpu(w, inp)
+    g = run_gpu(w, inp, fused=fused)
     assert m.moe_get_device_error(g["ws"]) == (0, 0)
     assert np.array_equal(to_np(g["ids"]), o["ids"])
     assert_gates_close(to_np(g["gates"]), o["gates"])
