@@ -7,9 +7,13 @@ One step is one pass of the whole path over one batch: moe_route, moe_layout
 (count + place kernels), moe_dispatch, moe_combine.  The expert FFN between
 dispatch and combine is not part of the path; its output y (the workload's
 stand-in expert applied to a warm-up dispatch of the same batch) is prepared
-before the timed region, like the inputs.  Between timed steps a 256 MiB
-buffer is written to flush the 126 MB L2; the flush sits outside the per-step
-CUDA events, and the step time is the sum of the event intervals.
+before the timed region, like the inputs.  L2 (126 MB): when the bytes one
+step touches exceed twice the L2 the steps run back to back (no step can find
+another's data in L2, and each step's dirty lines are written back during the
+next, which is the steady state); otherwise a 256 MiB buffer is written and
+then read between steps, outside the per-step CUDA events, so each step starts
+from an L2 holding only clean, unrelated lines.  The step time is the sum of
+the event intervals.
 
 Prints ONE JSON line (rank 0).  With N > 1 (torchrun, one process per GPU)
 every rank runs its own batch (weak scaling, no collective on the data path);
@@ -42,8 +46,9 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=200)
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--path", choices=["fused", "separate"], default="fused",
-                   help="route+layout as one moe_route_layout call, or two calls")
+    p.add_argument("--path", choices=["fused3", "fused", "separate"], default="fused3",
+                   help="steps 1-4 in one moe_route_layout_dispatch call; route+layout in one "
+                        "moe_route_layout call; or one call per step")
     return p.parse_args()
 
 
@@ -63,6 +68,7 @@ def algorithmic_bytes(w, kept_rows):
         + (T * row if w.shared else 0) + (T * row if w.residual else 0)
     # fused route + layout: the ids stay in the CTA between the two steps
     b["route_layout"] = b["route"] + b["layout"] - T * k * 4
+    b["route_layout_dispatch"] = b["route_layout"] + b["dispatch"] - T * k * 4
     return b
 
 
@@ -322,10 +328,34 @@ def main():
     kept_rows = int(lay.rank_counts.sum().item())
     m.moe_check(ws)
 
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    L2_BYTES = 126 * 10**6
+    touched = sum(algorithmic_bytes(w, kept_rows).values())
+    flush_between = touched < 2 * L2_BYTES
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush_between else None
+
+    def flush():
+        if flush_between:
+            flush_buf.fill_(1)
+            flush_buf.view(torch.int64).sum()  # read it back: L2 left clean
+
     stream = torch.cuda.current_stream(dev)
 
-    if args.path == "fused":
+    names_probe = ("route_layout", "dispatch", "combine")
+    ops_probe = (
+        lambda: m.moe_route_layout(shape, logits, bias, ws=ws, ids=ids, gates=gates, out=lay),
+        lambda: m.moe_dispatch(shape, x, lay.dst_pos, ws=ws, out=xd, scales=sc),
+        lambda: m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared,
+                              residual=residual, out=out),
+    )
+    if args.path == "fused3":
+        names = ("route_layout_dispatch", "combine")
+        ops = (
+            lambda: m.moe_route_layout_dispatch(shape, logits, x, bias, ws=ws, ids=ids, gates=gates,
+                                                lay=lay, out=xd, scales=sc),
+            lambda: m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared,
+                                  residual=residual, out=out),
+        )
+    elif args.path == "fused":
         names = ("route_layout", "dispatch", "combine")
         ops = (
             lambda: m.moe_route_layout(shape, logits, bias, ws=ws, ids=ids, gates=gates,
@@ -355,7 +385,7 @@ def main():
     side.wait_stream(stream)
     with torch.cuda.stream(side):
         for _ in range(max(3, args.warmup)):
-            flush.fill_(1)
+            flush()
             step()
     stream.wait_stream(side)
     torch.cuda.synchronize()
@@ -363,7 +393,7 @@ def main():
     with torch.cuda.graph(g_step):
         step()
     for _ in range(3):
-        flush.fill_(1)
+        flush()
         g_step.replay()
     torch.cuda.synchronize()
     m.moe_check(ws)
@@ -379,7 +409,7 @@ def main():
         sampler.start()
         time.sleep(0.3)
     for i in range(K):
-        flush.fill_(1)
+        flush()
         ev[i][0].record(stream)
         g_step.replay()
         ev[i][1].record(stream)
@@ -398,19 +428,21 @@ def main():
     # per-kernel breakdown: a probe graph of the same step with event-record
     # nodes between the kernels, replayed after an L2 flush and read back one
     # replay at a time
-    n_ops = len(ops)
+    probe_names = names if args.path != "fused3" else names_probe
+    probe_ops = ops if args.path != "fused3" else ops_probe
+    n_ops = len(probe_ops)
     probe_ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ops + 1)]
     g_probe = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_probe):
         cap = torch.cuda.current_stream(dev)
         probe_ev[0].record(cap)
-        for j, op in enumerate(ops):
+        for j, op in enumerate(probe_ops):
             op()
             probe_ev[j + 1].record(cap)
     K_ops = max(20, min(400, K // 10))
     sums = [0.0] * n_ops
     for i in range(K_ops):
-        flush.fill_(1)
+        flush()
         g_probe.replay()
         torch.cuda.synchronize()
         for j in range(n_ops):
@@ -453,13 +485,13 @@ def main():
     byts = algorithmic_bytes(w, kept_rows)
     peak, peak_kind = hbm_peak()
     kern = {}
-    for s, name in enumerate(names):
+    for s, name in enumerate(probe_names):
         us = mean[s] * 1e3
         gbs = byts[name] / (mean[s] * 1e-3) / 1e9
         kern[name] = {"us": round(us, 2), "bytes": byts[name], "gbs": round(gbs, 1),
                       "frac": round(gbs / peak, 4)}
-    t_disp = mean[names.index("dispatch")]
-    t_comb = mean[names.index("combine")]
+    t_disp = mean[probe_names.index("dispatch")]
+    t_comb = mean[probe_names.index("combine")]
     dom = "dispatch" if t_disp >= t_comb else "combine"
     dom_gbs = byts[dom] / (max(t_disp, t_comb) * 1e-3) / 1e9
     dc_ms = t_disp + t_comb
@@ -481,7 +513,10 @@ def main():
         "config": {"workload": w.describe(), "tokens": T, "hidden": w.H, "experts": w.E,
                    "k": k, "ranks": w.R, "capacity": w.capacity, "rows": N,
                    "kept_rows": kept_rows, "parallelism": f"replicas x{world}",
-                   "l2": "256 MiB write between timed steps, outside the step events",
+                   "l2": ("256 MiB write + read between timed steps, outside the step events"
+                          if flush_between else
+                          f"no flush: inputs larger than L2 ({touched / 1e6:.0f} MB touched per "
+                          f"step vs 126 MB L2), steps back to back"),
                    "step": " + ".join(names) + ", one CUDA graph"},
         "dispatch_combine": {"tokens_per_s": world * T / (dc_ms * 1e-3),
                              "us": round(dc_ms * 1e3, 2), "gbs": round(dc_gbs, 1),
@@ -492,7 +527,7 @@ def main():
                      "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
                      "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
                      "traffic": ncu_traffic(dom, w.name)},
-        "gpu_launches": len(ops) * K,
+        "gpu_launches": {"fused3": 4, "fused": 4, "separate": 5}[args.path] * K,
         "clocks": clocks,
         "e2e": e2e,
     }

@@ -27,7 +27,7 @@ from . import _binding
 from ._binding import MoeError, MOE_F_FP8, MOE_F_RENORM
 
 __all__ = ["MoeShape", "Workspace", "Layout", "MoeError", "moe_route", "moe_layout",
-           "moe_route_layout",
+           "moe_route_layout", "moe_route_layout_dispatch",
            "moe_dispatch", "moe_combine", "moe_get_device_error", "moe_check",
            "moe_layout_rows", "moe_workspace_bytes"]
 
@@ -186,6 +186,55 @@ def moe_route_layout(shape: MoeShape, logits: torch.Tensor, bias: Optional[torch
         _ptr(out.src_idx, "src_idx", torch.int32, (N,)), ws.ptr, ws.nbytes, _stream(dev))
     _check(st, "moe_route_layout")
     return ids, gates, out
+
+
+def _dispatch_out(shape: MoeShape, dev, out, scales):
+    N, H = shape.rows, shape.hidden
+    if shape.fp8:
+        if out is None:
+            out = torch.empty((N, H), dtype=torch.float8_e4m3fn, device=dev)
+        if scales is None:
+            scales = torch.empty((N, H // 128), dtype=torch.float32, device=dev)
+        return out, scales, _ptr(out, "out", torch.float8_e4m3fn, (N, H)), \
+            _ptr(scales, "scales", torch.float32, (N, H // 128))
+    if out is None:
+        out = torch.empty((N, H), dtype=torch.bfloat16, device=dev)
+    return out, None, _ptr(out, "out", torch.bfloat16, (N, H)), None
+
+
+def moe_route_layout_dispatch(shape: MoeShape, logits: torch.Tensor, x: torch.Tensor,
+                              bias: Optional[torch.Tensor] = None, *, ws: Workspace,
+                              ids: Optional[torch.Tensor] = None,
+                              gates: Optional[torch.Tensor] = None, lay: Optional[Layout] = None,
+                              out: Optional[torch.Tensor] = None,
+                              scales: Optional[torch.Tensor] = None):
+    """Steps 1-4 in one call.  Returns (ids, gates, Layout, dispatched) where
+    dispatched is as moe_dispatch returns it."""
+    T, E, k, R, H = shape.tokens, shape.experts, shape.k, shape.ranks, shape.hidden
+    N = shape.rows
+    dev = logits.device
+    i32 = dict(dtype=torch.int32, device=dev)
+    if ids is None:
+        ids = torch.empty((T, k), **i32)
+    if gates is None:
+        gates = torch.empty((T, k), dtype=torch.float32, device=dev)
+    if lay is None:
+        lay = Layout(torch.empty(E, **i32), torch.empty(E + 1, **i32), torch.empty(R + 1, **i32),
+                     torch.empty(R, **i32), torch.empty((T, k), **i32), torch.empty(N, **i32))
+    out, scales, optr, sptr = _dispatch_out(shape, dev, out, scales)
+    st = _binding.lib().moe_route_layout_dispatch(
+        ctypes.byref(shape.c()), _ptr(logits, "logits", torch.float32, (T, E)),
+        _ptr(bias, "bias", torch.float32, (E,)), _ptr(x, "x", torch.bfloat16, (T, H)),
+        _ptr(ids, "ids", torch.int32, (T, k)), _ptr(gates, "gates", torch.float32, (T, k)),
+        _ptr(lay.counts, "counts", torch.int32, (E,)),
+        _ptr(lay.expert_off, "expert_off", torch.int32, (E + 1,)),
+        _ptr(lay.rank_off, "rank_off", torch.int32, (R + 1,)),
+        _ptr(lay.rank_counts, "rank_counts", torch.int32, (R,)),
+        _ptr(lay.dst_pos, "dst_pos", torch.int32, (T, k)),
+        _ptr(lay.src_idx, "src_idx", torch.int32, (N,)), optr, sptr, ws.ptr, ws.nbytes,
+        _stream(dev))
+    _check(st, "moe_route_layout_dispatch")
+    return ids, gates, lay, ((out, scales) if shape.fp8 else out)
 
 
 def moe_dispatch(shape: MoeShape, x: torch.Tensor, dst_pos: torch.Tensor, *, ws: Workspace,

@@ -28,6 +28,7 @@ EXPORTS = (
     "moe_abi_version", "moe_status_string", "moe_layout_rows", "moe_workspace_bytes",
     "moe_workspace_init", "moe_route", "moe_layout", "moe_dispatch", "moe_combine",
     "moe_get_device_error", "moe_layout_noalloc", "moe_route_layout",
+    "moe_route_layout_dispatch",
 )
 
 
@@ -74,6 +75,9 @@ def lib(path: str = None):
     L.moe_layout.restype = i32
     L.moe_route_layout.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.moe_route_layout.restype = i32
+    L.moe_route_layout_dispatch.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                            vp, sz, vp]
+    L.moe_route_layout_dispatch.restype = i32
     L.moe_dispatch.argtypes = [sp, vp, vp, vp, vp, vp, sz, vp]
     L.moe_dispatch.restype = i32
     L.moe_combine.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, sz, vp]

@@ -12,7 +12,6 @@ namespace {
 
 using moe::WsHeader;
 
-constexpr uint64_t kLayoutTimeoutNs = 1000000000ull;  // bounded lookback wait: 1 s
 constexpr size_t kHeaderBytes = sizeof(WsHeader);
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -40,15 +39,13 @@ int64_t rows_of(const moe_shape_t* s) {
                          : int64_t(s->tokens) * s->k + int64_t(s->experts) * (s->align - 1);
 }
 
-int64_t tiles_of(const moe_shape_t* s) {
-  const int64_t T = s->tokens;
-  return T > 0 ? (T + moe::kLayoutTileTokens - 1) / moe::kLayoutTileTokens : 1;
+// Workspace: header, then two tile tables of equal size (words a multiple of 4).
+size_t ws_bytes_of(const moe_shape_t* s) {
+  const size_t words = (moe::layout_table_words(s->tokens, s->experts) + 3) / 4 * 4;
+  return kHeaderBytes + 2 * words * sizeof(uint32_t);
 }
 
-size_t ws_bytes_of(const moe_shape_t* s) {
-  const size_t table = size_t(tiles_of(s)) * size_t(s->experts) * sizeof(uint32_t);
-  return kHeaderBytes + ((table + 255) / 256) * 256;
-}
+size_t half_words_of(size_t ws_bytes) { return ((ws_bytes - kHeaderBytes) / 8) / 4 * 4; }
 
 moe_status_t ws_ok(const moe_shape_t* s, void* ws, size_t ws_bytes) {
   if (ws == nullptr || !aligned(ws, 16)) return MOE_ERR_WORKSPACE;
@@ -146,11 +143,11 @@ moe_status_t moe_layout(const moe_shape_t* shape, const int32_t* ids, int32_t* c
   moe_status_t st = ws_ok(shape, ws, ws_bytes);
   if (st != MOE_OK) return st;
   WsHeader* hdr = static_cast<WsHeader*>(ws);
-  uint32_t* table = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + kHeaderBytes);
+  uint32_t* tables = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + kHeaderBytes);
   return from_cuda(moe::launch_layout(env_of(stream), ids, shape->tokens, shape->experts,
                                       shape->k, shape->ranks, shape->capacity, shape->align, N,
-                                      table, hdr, counts, expert_off, rank_off, rank_counts,
-                                      dst_pos, src_idx, kLayoutTimeoutNs));
+                                      tables, half_words_of(ws_bytes), hdr, counts, expert_off,
+                                      rank_off, rank_counts, dst_pos, src_idx, true));
 }
 
 moe_status_t moe_route_layout(const moe_shape_t* shape, const float* logits, const float* bias,
@@ -173,12 +170,44 @@ moe_status_t moe_route_layout(const moe_shape_t* shape, const float* logits, con
   moe_status_t st = ws_ok(shape, ws, ws_bytes);
   if (st != MOE_OK) return st;
   WsHeader* hdr = static_cast<WsHeader*>(ws);
-  uint32_t* table = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + kHeaderBytes);
-  return from_cuda(moe::launch_route_layout(
-      env_of(stream), logits, bias, (shape->flags & MOE_F_RENORM) ? 1 : 0, ids, gates,
-      shape->tokens, shape->experts, shape->k, shape->ranks, shape->capacity, shape->align, N,
-      table, hdr, counts, expert_off, rank_off, rank_counts, dst_pos, src_idx,
-      kLayoutTimeoutNs));
+  uint32_t* tables = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + kHeaderBytes);
+  const size_t half = half_words_of(ws_bytes);
+  const moe::LaunchEnv env = env_of(stream);
+  if (shape->tokens > 0) {
+    const cudaError_t err = moe::launch_route(env, logits, bias, shape->tokens, shape->experts,
+                                              shape->k, (shape->flags & MOE_F_RENORM) ? 1 : 0,
+                                              ids, gates, hdr, tables, half);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return from_cuda(moe::launch_layout(env, ids, shape->tokens, shape->experts, shape->k,
+                                      shape->ranks, shape->capacity, shape->align, N, tables, half,
+                                      hdr, counts, expert_off, rank_off, rank_counts, dst_pos,
+                                      src_idx, false));
+}
+
+moe_status_t moe_route_layout_dispatch(const moe_shape_t* shape, const float* logits,
+                                       const float* bias, const void* x, int32_t* ids,
+                                       float* gates, int32_t* counts, int32_t* expert_off,
+                                       int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
+                                       int32_t* src_idx, void* out, float* scales, void* ws,
+                                       size_t ws_bytes, moe_stream_t stream) {
+  if (!shape_ok(shape)) return MOE_ERR_INVALID_ARG;
+  const bool fp8 = (shape->flags & MOE_F_FP8) != 0u;
+  if (shape->tokens > 0 && (x == nullptr || out == nullptr || (fp8 && scales == nullptr)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(out, 16) || !aligned(scales, 4)) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = moe_route_layout(shape, logits, bias, ids, gates, counts, expert_off,
+                                     rank_off, rank_counts, dst_pos, src_idx, ws, ws_bytes,
+                                     stream);
+  if (st != MOE_OK || shape->tokens == 0) return st;
+  const moe::LaunchEnv env = env_of(stream);
+  WsHeader* hdr = static_cast<WsHeader*>(ws);
+  const int64_t N = rows_of(shape);
+  if (fp8)
+    return from_cuda(moe::launch_dispatch_fp8(env, x, dst_pos, shape->tokens, shape->hidden,
+                                              shape->k, N, out, scales, hdr));
+  return from_cuda(moe::launch_dispatch_bf16(env, x, dst_pos, shape->tokens, shape->hidden,
+                                             shape->k, N, out, hdr, true));
 }
 
 moe_status_t moe_dispatch(const moe_shape_t* shape, const void* x, const int32_t* dst_pos,

@@ -9,11 +9,11 @@
 // section "Why the router can ruin your day": a dropped slot counts as if the
 // token skipped that expert.
 //
-// Token-major gather, HBM-bound.  A token row is split over G threads of CPT
-// 16-byte chunks; each thread issues the loads of up to kBatch slots before
-// using any of them (independent 16-byte loads in flight), then accumulates
-// in fp32 in slot order j = 0..k-1 with explicit round-to-nearest FMAs, adds
-// the shared-expert row and the residual row, and rounds to bf16 once.
+// Token-major gather, HBM-bound.  Each warp owns a 32*CPT-chunk slice of one
+// token row; each lane issues the 16-byte loads of up to kBatch slots before
+// using any of them (independent loads in flight), then accumulates in fp32
+// in slot order j = 0..k-1 with explicit round-to-nearest FMAs, adds the
+// shared-expert row and the residual row, and rounds to bf16 once.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -24,7 +24,8 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kBatch = 8;
+constexpr int kBatch = 4;     // slots whose loads are in flight together
+constexpr int kMinBlocks = 4;  // CTAs per SM the register budget must allow
 
 __device__ __forceinline__ void fma8(float (&acc)[8], float g, const uint4& v) {
   acc[0] = __fmaf_rn(g, bf16lo(v.x), acc[0]);
@@ -53,51 +54,57 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// One warp per (token, slice of 32*CPT chunks); lane j < k fetches the row
+// and gate of slot j once and the warp broadcasts them by shuffle.
 template <int CPT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, kMinBlocks)
     combine_kernel(const char* __restrict__ y, const int32_t* __restrict__ dst_pos,
                    const float* __restrict__ gates, const char* __restrict__ shared,
                    const char* __restrict__ residual, int T, int H, int k, int64_t N,
                    char* __restrict__ out, WsHeader* hdr) {
+  pdl_wait();  // y, gates and dst_pos may come from the kernel launched just before
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
   const int C8 = H >> 3;
-  const int G = (C8 + CPT - 1) / CPT;
-  const int64_t units = (int64_t)T * G;
+  const int S = (C8 + 32 * CPT - 1) / (32 * CPT);
+  const int64_t tasks = (int64_t)T * S;
   const size_t row_bytes = (size_t)H * 2;
-  for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < units;
-       u += (int64_t)gridDim.x * kThreads) {
-    const int t = (int)(u / G);
-    const int g = (int)(u - (int64_t)t * G);
+  const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
+  for (int64_t task = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5; task < tasks;
+       task += nw) {
+    const int t = (int)(task / S);
+    const int cb = (int)(task - (int64_t)t * S) * 32 * CPT + lane;
+    int pl = -1;
+    float gl = 0.0f;
+    if (lane < k) {
+      pl = __ldg(dst_pos + (size_t)t * k + lane);
+      gl = __ldg(gates + (size_t)t * k + lane);
+      if (pl >= N) {
+        report(hdr, MOE_ERR_DEVICE_RANGE, pl);
+        pl = -1;
+      }
+    }
     float acc[CPT][8];
 #pragma unroll
     for (int i = 0; i < CPT; ++i)
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[i][e] = 0.0f;
 
-    const int32_t* dp = dst_pos + (size_t)t * k;
-    const float* gp = gates + (size_t)t * k;
     for (int j0 = 0; j0 < k; j0 += kBatch) {
       uint4 v[kBatch][CPT];
       float gw[kBatch];
-      bool use[kBatch];
+      int pp[kBatch];
 #pragma unroll
       for (int jj = 0; jj < kBatch; ++jj) {
-        const int j = j0 + jj;
-        int p = -1;
-        gw[jj] = 0.0f;
-        if (j < k) {
-          p = __ldg(dp + j);
-          gw[jj] = __ldg(gp + j);
-          if (p >= N) {
-            if (g == 0) report(hdr, MOE_ERR_DEVICE_RANGE, p);
-            p = -1;
-          }
-        }
-        use[jj] = p >= 0;
-        const char* src = y + (size_t)(p < 0 ? 0 : p) * row_bytes;
+        const int j = j0 + jj;  // j < 32: the shuffle source is always a lane
+        pp[jj] = __shfl_sync(kFull, pl, j & 31);
+        gw[jj] = __shfl_sync(kFull, gl, j & 31);
+        if (j >= k) pp[jj] = -1;
+        const char* src = y + (size_t)(pp[jj] < 0 ? 0 : pp[jj]) * row_bytes;
 #pragma unroll
         for (int i = 0; i < CPT; ++i) {
-          const int c = g + i * G;
-          if (use[jj] && c < C8)
+          const int c = cb + 32 * i;
+          if (pp[jj] >= 0 && c < C8)
             v[jj][i] = ld16_stream(src + (size_t)c * 16);
           else
             v[jj][i] = make_uint4(0, 0, 0, 0);
@@ -105,7 +112,7 @@ __global__ void __launch_bounds__(kThreads)
       }
 #pragma unroll
       for (int jj = 0; jj < kBatch; ++jj)
-        if (use[jj]) {
+        if (pp[jj] >= 0) {
 #pragma unroll
           for (int i = 0; i < CPT; ++i) fma8(acc[i], gw[jj], v[jj][i]);
         }
@@ -113,7 +120,7 @@ __global__ void __launch_bounds__(kThreads)
 
 #pragma unroll
     for (int i = 0; i < CPT; ++i) {
-      const int c = g + i * G;
+      const int c = cb + 32 * i;
       if (c >= C8) continue;
       const size_t off = (size_t)t * row_bytes + (size_t)c * 16;
       if (shared != nullptr) add8(acc[i], ld16_stream(shared + off));
@@ -148,11 +155,10 @@ cudaError_t launch_combine(const LaunchEnv& env, const void* y, const int32_t* d
   if (T == 0) return cudaSuccess;
   const int C8 = H / 8;
   auto kern = combine_kernel<1>;
-  const int grid = grid_for(kern, env, (int64_t)T * C8);
-  kern<<<grid, kThreads, 0, env.stream>>>(
-      static_cast<const char*>(y), dst_pos, gates, static_cast<const char*>(shared),
-      static_cast<const char*>(residual), T, H, k, N, static_cast<char*>(out), hdr);
-  return cudaGetLastError();
+  const int grid = grid_for(kern, env, (int64_t)T * ((C8 + 31) / 32) * 32);
+  return launch_pdl(env, kern, dim3(grid), dim3(kThreads), 0, static_cast<const char*>(y), dst_pos,
+                    gates, static_cast<const char*>(shared), static_cast<const char*>(residual), T,
+                    H, k, N, static_cast<char*>(out), hdr);
 }
 
 }  // namespace moe

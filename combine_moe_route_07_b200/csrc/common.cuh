@@ -13,12 +13,13 @@ constexpr unsigned kFull = 0xffffffffu;
 
 // Workspace header (first 256 bytes of every workspace).
 struct WsHeader {
-  int32_t err;            // first device-side error code (moe_status_t), 0 = none
-  int32_t detail;         // index that caused it
-  uint32_t looked;        // layout: tiles whose lookback is done
-  uint32_t totals_ready;  // layout: expert offsets are published
-  uint32_t finished;      // layout: tiles that are done; the last one resets the three
-  uint32_t pad[59];
+  int32_t err;             // first device-side error code (moe_status_t), 0 = none
+  int32_t detail;          // index that caused it
+  uint32_t reserved[2];
+  uint32_t epoch;          // layout: which of the two tile tables the next call fills
+  uint32_t done;           // layout: place CTAs finished (the last one bumps epoch)
+  uint32_t words_used[2];  // layout: words of each table filled since it was last cleared
+  uint32_t pad[56];        // (epoch..words_used form one 16-byte word at offset 16)
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 
@@ -51,6 +52,15 @@ __device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
 }
 // L2-coherent 32-bit load (bypasses L1), for data another CTA published.
 __device__ __forceinline__ int32_t ld_cg(const int32_t* p) { return __ldcg(p); }
+
+// Programmatic dependent launch.  pdl_wait(): block until the kernel this one
+// was launched behind has finished and its writes are visible (returns at once
+// when launched without the attribute).  pdl_trigger(): allow the kernel
+// launched behind this one to start placing its CTAs.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;

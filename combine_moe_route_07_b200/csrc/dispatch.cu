@@ -8,17 +8,17 @@
 // them anyway.
 //
 // Token-major and HBM-bound: no step is a contraction, so the kernel is a
-// streaming copy.  A token row is split over G threads; each thread holds
-// CPT 16-byte chunks (chunks g, g+G, ... so a warp touches contiguous
-// 512-byte runs), loads them once with L1-bypassing loads and issues k
-// 16-byte stores per chunk.  Grid: a whole number of waves of resident CTAs.
+// streaming copy.  Each warp loads a 32*CPT-chunk slice of one token row once
+// (16-byte L1-bypassing loads) and issues k 16-byte stores per chunk.  Grid:
+// the CTAs that fit on the GPU at once, striding over (token, slice) tasks.
 //
-// FP8 variant: the 16 chunks of a 128-channel block sit in 16 aligned lanes;
-// amax is a 4-step xor shuffle, then scale = amax/448, inv = 448/amax (IEEE
-// division), codes = cvt.rn.satfinite.e4m3x2(x * inv) and 8-byte stores.
+// FP8 variant: per 128-channel block, amax by xor shuffle, scale = amax/448,
+// inv = 448/amax (IEEE division), codes = cvt.rn.satfinite.e4m3x2(x * inv),
+// 8-byte stores.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include "bulk.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -28,39 +28,140 @@ namespace {
 
 constexpr int kThreads = 256;
 
+// One warp per (token, slice of 32*CPT chunks): lane l holds chunks
+// slice*32*CPT + l + 32*i, so each warp load or store is one contiguous 512 B
+// run.  Lane j < k fetches dst_pos[t][j] once; the rows are broadcast by shuffle.
 template <int CPT>
 __global__ void __launch_bounds__(kThreads)
     dispatch_bf16_kernel(const char* __restrict__ x, const int32_t* __restrict__ dst_pos, int T,
                          int H, int k, int64_t N, char* __restrict__ out, WsHeader* hdr) {
+  pdl_wait();  // x and dst_pos may come from the kernel launched just before
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
   const int C8 = H >> 3;  // 16-byte chunks per row
-  const int G = (C8 + CPT - 1) / CPT;
-  const int64_t units = (int64_t)T * G;
+  const int S = (C8 + 32 * CPT - 1) / (32 * CPT);
+  const int64_t tasks = (int64_t)T * S;
   const size_t row_bytes = (size_t)H * 2;
-  for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < units;
-       u += (int64_t)gridDim.x * kThreads) {
-    const int t = (int)(u / G);
-    const int g = (int)(u - (int64_t)t * G);
+  const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
+  for (int64_t task = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5; task < tasks;
+       task += nw) {
+    const int t = (int)(task / S);
+    const int cb = (int)(task - (int64_t)t * S) * 32 * CPT + lane;
     const char* src = x + (size_t)t * row_bytes;
     uint4 v[CPT];
 #pragma unroll
     for (int i = 0; i < CPT; ++i) {
-      const int c = g + i * G;
+      const int c = cb + 32 * i;
       if (c < C8) v[i] = ld16_stream(src + (size_t)c * 16);
     }
-    const int32_t* dp = dst_pos + (size_t)t * k;
+    const int pl = lane < k ? __ldg(dst_pos + (size_t)t * k + lane) : -1;
     for (int j = 0; j < k; ++j) {
-      const int p = __ldg(dp + j);
+      const int p = __shfl_sync(kFull, pl, j);
       if (p < 0) continue;
       if (p >= N) {
-        if (g == 0) report(hdr, MOE_ERR_DEVICE_RANGE, p);
+        if (lane == 0) report(hdr, MOE_ERR_DEVICE_RANGE, p);
         continue;
       }
       char* dst = out + (size_t)p * row_bytes;
 #pragma unroll
       for (int i = 0; i < CPT; ++i) {
-        const int c = g + i * G;
+        const int c = cb + 32 * i;
         if (c < C8) st16(dst + (size_t)c * 16, v[i]);
       }
+    }
+  }
+}
+
+// Bulk-copy (TMA) variant for rows of 1-32 KiB.  Each CTA runs kBulkWarps
+// independent pipelines; lane 0 of a warp streams its tokens through
+// `stages` shared-memory row buffers: a bulk load global -> shared completes
+// on the stage's mbarrier, then k bulk stores shared -> global (one bulk
+// group per token) write the copies, and the stage is refilled once the
+// previous token's group has finished reading it.  No thread touches the row
+// data, so the LSU carries only the dst_pos loads.  Every wait is bounded.
+constexpr int kBulkWarps = 4;
+constexpr int kBulkMaxStages = 8;
+constexpr uint64_t kBulkTimeoutNs = 1000000000ull;
+
+__global__ void __launch_bounds__(kBulkWarps * 32)
+    dispatch_bf16_bulk_kernel(const char* __restrict__ x, const int32_t* __restrict__ dst_pos,
+                              int T, int H, int k, int64_t N, char* __restrict__ out, int stages,
+                              uint32_t stage_bytes, int x_ready, WsHeader* hdr) {
+  extern __shared__ __align__(128) unsigned char sbuf[];
+  __shared__ uint64_t bars[kBulkWarps][kBulkMaxStages];
+  // x_ready: the kernel launched just before this one did not write x, and
+  // every kernel before it has finished (true behind this library's own route
+  // and layout kernels, which each wait for their predecessor before letting
+  // the next start), so the first rows can be fetched before the wait below.
+  if (!x_ready) {
+    pdl_wait();  // x and dst_pos may come from the kernel launched just before
+    pdl_trigger();
+  }
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t row = (uint32_t)H * 2u;
+  unsigned char* st = sbuf + (size_t)w * stages * stage_bytes;
+  uint64_t* bar = bars[w];
+  if (lane == 0) {
+    for (int s = 0; s < stages; ++s) mbar_init(&bar[s], 1);
+    mbar_fence_init();
+  }
+  __syncwarp();
+  const int64_t stride = (int64_t)gridDim.x * kBulkWarps;
+  const int64_t first = (int64_t)blockIdx.x * kBulkWarps + w;
+  const int64_t count = first < T ? (T - 1 - first) / stride + 1 : 0;
+  int64_t issued = 0;  // loads issued (lane 0)
+  if (lane == 0) {
+    for (; issued < count && issued < stages - 1; ++issued) {
+      mbar_arrive_expect_tx(&bar[issued], row);
+      bulk_load(st + (size_t)issued * stage_bytes, x + (size_t)(first + issued * stride) * row,
+                row, &bar[issued]);
+    }
+  }
+  if (x_ready) {  // dst_pos comes from the kernel launched just before
+    pdl_wait();
+    pdl_trigger();
+  }
+  uint32_t parity = 0;  // bit s: the phase stage s completes next
+  bool ok = true;
+  int pl = (count > 0 && lane < k) ? __ldg(dst_pos + (size_t)first * k + lane) : -1;
+  for (int64_t i = 0; i < count && ok; ++i) {
+    const int s = (int)(i % stages);
+    const int p_cur = pl;
+    if (i + 1 < count && lane < k)  // next token's rows, while this one streams
+      pl = __ldg(dst_pos + (size_t)(first + (i + 1) * stride) * k + lane);
+    if (lane == 0) {
+      ok = mbar_wait_bounded(&bar[s], (parity >> s) & 1u, kBulkTimeoutNs);
+      parity ^= 1u << s;
+      if (!ok) report(hdr, MOE_ERR_DEVICE_TIMEOUT, (int)(first + i * stride));
+    }
+    ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
+    if (!ok) break;
+    for (int j = 0; j < k; ++j) {
+      const int p = __shfl_sync(kFull, p_cur, j);
+      if (lane == 0 && p >= 0) {
+        if (p < N)
+          bulk_store(out + (size_t)p * row, st + (size_t)s * stage_bytes, row);
+        else
+          report(hdr, MOE_ERR_DEVICE_RANGE, p);
+      }
+    }
+    if (lane == 0) {
+      bulk_commit();
+      if (issued < count) {  // refill the stage token i-1 used
+        bulk_wait_read<1>();
+        const int sn = (int)(issued % stages);
+        mbar_arrive_expect_tx(&bar[sn], row);
+        bulk_load(st + (size_t)sn * stage_bytes, x + (size_t)(first + issued * stride) * row, row,
+                  &bar[sn]);
+        ++issued;
+      }
+    }
+    __syncwarp();
+  }
+  if (lane == 0) {
+    bulk_wait_all();
+    if (!ok) {  // let the loads still in flight land before the CTA exits
+      for (int s = 0; s < stages; ++s) (void)mbar_wait_bounded(&bar[s], (parity >> s) & 1u, kBulkTimeoutNs);
     }
   }
 }
@@ -73,35 +174,35 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
   return (uint32_t)lo | ((uint32_t)hi << 16);
 }
 
-// G is a multiple of 16 so that the 16 threads of a 128-channel block are 16
-// aligned lanes of one warp.  The loop runs per warp (all lanes iterate
-// together) because the amax reduction shuffles across the block's lanes.
+// Same warp-per-(token, slice) mapping; the 16 chunks of a 128-channel
+// block are 16 aligned lanes (slices start at multiples of 32 chunks), so the
+// block's amax is a 4-step xor shuffle inside each half-warp.
 template <int CPT>
 __global__ void __launch_bounds__(kThreads)
     dispatch_fp8_kernel(const char* __restrict__ x, const int32_t* __restrict__ dst_pos, int T,
                         int H, int k, int64_t N, uint8_t* __restrict__ out,
                         float* __restrict__ scales, WsHeader* hdr) {
-  const int C8 = H >> 3;
-  const int G = (((C8 + CPT - 1) / CPT) + 15) & ~15;
-  const int nb = H >> 7;  // scale blocks per row
-  const int64_t units = (int64_t)T * G;
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
+  const int C8 = H >> 3;
+  const int S = (C8 + 32 * CPT - 1) / (32 * CPT);
+  const int nb = H >> 7;  // scale blocks per row
+  const int64_t tasks = (int64_t)T * S;
   const size_t row_bytes = (size_t)H * 2;
-  const int64_t warp0 = ((int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31));
-  for (int64_t ub = warp0; ub < units; ub += (int64_t)gridDim.x * kThreads) {
-    const int64_t u = ub + lane;
-    const bool live = u < units;
-    const int t = live ? (int)(u / G) : 0;
-    const int g = live ? (int)(u - (int64_t)t * G) : 0;
+  const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
+  for (int64_t task = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5; task < tasks;
+       task += nw) {
+    const int t = (int)(task / S);
+    const int cb = (int)(task - (int64_t)t * S) * 32 * CPT + lane;
     const char* src = x + (size_t)t * row_bytes;
     uint32_t q[CPT][2];
     float s[CPT];
 #pragma unroll
     for (int i = 0; i < CPT; ++i) {
-      const int c = g + i * G;
-      const bool in = live && c < C8;
+      const int c = cb + 32 * i;
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (in) v = ld16_stream(src + (size_t)c * 16);
+      if (c < C8) v = ld16_stream(src + (size_t)c * 16);
       float f[8] = {bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y),
                     bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w)};
       float amax = 0.0f;
@@ -122,20 +223,19 @@ __global__ void __launch_bounds__(kThreads)
         q[i][1] = 0u;
       }
     }
-    if (!live) continue;
-    const int32_t* dp = dst_pos + (size_t)t * k;
+    const int pl = lane < k ? __ldg(dst_pos + (size_t)t * k + lane) : -1;
     for (int j = 0; j < k; ++j) {
-      const int p = __ldg(dp + j);
+      const int p = __shfl_sync(kFull, pl, j);
       if (p < 0) continue;
       if (p >= N) {
-        if (g == 0) report(hdr, MOE_ERR_DEVICE_RANGE, p);
+        if (lane == 0) report(hdr, MOE_ERR_DEVICE_RANGE, p);
         continue;
       }
       uint8_t* dst = out + (size_t)p * H;
       float* sdst = scales + (size_t)p * nb;
 #pragma unroll
       for (int i = 0; i < CPT; ++i) {
-        const int c = g + i * G;
+        const int c = cb + 32 * i;
         if (c < C8) {
           *reinterpret_cast<uint2*>(dst + (size_t)c * 8) = make_uint2(q[i][0], q[i][1]);
           if ((c & 15) == 0) sdst[c >> 4] = s[i];
@@ -160,21 +260,44 @@ int grid_for(K kernel, const LaunchEnv& env, int64_t units) {
 }  // namespace
 
 cudaError_t launch_dispatch_bf16(const LaunchEnv& env, const void* x, const int32_t* dst_pos,
-                                 int T, int H, int k, int64_t N, void* out, WsHeader* hdr) {
+                                 int T, int H, int k, int64_t N, void* out, WsHeader* hdr,
+                                 bool x_ready) {
   if (T == 0) return cudaSuccess;
   const int C8 = H / 8;
   const char* xs = static_cast<const char*>(x);
   char* o = static_cast<char*>(out);
-  if (C8 >= 512) {
+  const uint32_t row = (uint32_t)H * 2u;
+  if (row >= 1024 && row <= 32768) {
+    const uint32_t stage_bytes = (row + 127u) & ~127u;
+    int stages = (int)((200u * 1024u) / (kBulkWarps * stage_bytes));
+    if (stages > kBulkMaxStages) stages = kBulkMaxStages;
+    if (stages >= 2) {
+      const size_t smem = (size_t)kBulkWarps * stages * stage_bytes;
+      cudaError_t err = cudaFuncSetAttribute(dispatch_bf16_bulk_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (err != cudaSuccess) return err;
+      int per_sm = 0;
+      err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dispatch_bf16_bulk_kernel,
+                                                          kBulkWarps * 32, smem);
+      if (err != cudaSuccess) return err;
+      if (per_sm < 1) per_sm = 1;
+      int64_t grid = (int64_t)per_sm * env.num_sms;
+      const int64_t need = ((int64_t)T + kBulkWarps - 1) / kBulkWarps;
+      if (grid > need) grid = need;
+      return launch_pdl(env, dispatch_bf16_bulk_kernel, dim3((unsigned)grid),
+                        dim3(kBulkWarps * 32), smem, xs, dst_pos, T, H, k, N, o, stages,
+                        stage_bytes, x_ready ? 1 : 0, hdr);
+    }
+  }
+  if (C8 >= 256) {
     auto kern = dispatch_bf16_kernel<2>;
-    const int grid = grid_for(kern, env, (int64_t)T * ((C8 + 1) / 2));
-    kern<<<grid, kThreads, 0, env.stream>>>(xs, dst_pos, T, H, k, N, o, hdr);
+    const int grid = grid_for(kern, env, (int64_t)T * ((C8 + 63) / 64) * 32);
+    return launch_pdl(env, kern, dim3(grid), dim3(kThreads), 0, xs, dst_pos, T, H, k, N, o, hdr);
   } else {
     auto kern = dispatch_bf16_kernel<1>;
-    const int grid = grid_for(kern, env, (int64_t)T * C8);
-    kern<<<grid, kThreads, 0, env.stream>>>(xs, dst_pos, T, H, k, N, o, hdr);
+    const int grid = grid_for(kern, env, (int64_t)T * ((C8 + 31) / 32) * 32);
+    return launch_pdl(env, kern, dim3(grid), dim3(kThreads), 0, xs, dst_pos, T, H, k, N, o, hdr);
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_dispatch_fp8(const LaunchEnv& env, const void* x, const int32_t* dst_pos,
@@ -183,11 +306,9 @@ cudaError_t launch_dispatch_fp8(const LaunchEnv& env, const void* x, const int32
   if (T == 0) return cudaSuccess;
   const int C8 = H / 8;
   auto kern = dispatch_fp8_kernel<1>;
-  const int G = (C8 + 15) & ~15;
-  const int grid = grid_for(kern, env, (int64_t)T * G);
-  kern<<<grid, kThreads, 0, env.stream>>>(static_cast<const char*>(x), dst_pos, T, H, k, N,
-                                          static_cast<uint8_t*>(out), scales, hdr);
-  return cudaGetLastError();
+  const int grid = grid_for(kern, env, (int64_t)T * ((C8 + 31) / 32) * 32);
+  return launch_pdl(env, kern, dim3(grid), dim3(kThreads), 0, static_cast<const char*>(x), dst_pos,
+                    T, H, k, N, static_cast<uint8_t*>(out), scales, hdr);
 }
 
 }  // namespace moe

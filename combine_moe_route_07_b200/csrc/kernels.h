@@ -14,28 +14,74 @@ struct LaunchEnv {
   int num_sms;
 };
 
-// Tokens per layout tile (one CTA per tile); the launch doubles it while the
-// tiles outnumber the CTAs that fit on the GPU at once.
-constexpr int kLayoutTileTokens = 128;
+// Launch `kernel` on env.stream with programmatic stream serialization, so
+// its CTAs may start while the previous kernel drains (the kernel calls
+// pdl_wait() before touching anything the previous kernel wrote).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(const LaunchEnv& env, void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                       size_t smem, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = env.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
+// Layout tiles: runs of TT consecutive tokens, TT a multiple of
+// kLayoutTileQuantum, at most kLayoutMaxTiles of them.  The workspace holds
+// two tables (used on alternate calls) of one row of E counters per tile.
+constexpr int kLayoutTileQuantum = 16;
+constexpr int kLayoutMaxTiles = 128;
+
+struct TileGeom {
+  int TT;  // tokens per tile
+  int G;   // tiles
+};
+inline TileGeom layout_tiles(int T) {
+  TileGeom g;
+  const int64_t q = kLayoutTileQuantum;
+  int64_t want = T > 0 ? (T + q - 1) / q : 1;
+  if (want > kLayoutMaxTiles) want = kLayoutMaxTiles;
+  int64_t tt = T > 0 ? (T + want - 1) / want : q;
+  tt = ((tt + q - 1) / q) * q;
+  g.TT = (int)tt;
+  g.G = T > 0 ? (int)((T + tt - 1) / tt) : 1;
+  return g;
+}
+// Words in one of the two tile tables for T tokens and E experts.
+inline size_t layout_table_words(int T, int E) {
+  int64_t rows = T > 0 ? ((int64_t)T + kLayoutTileQuantum - 1) / kLayoutTileQuantum : 1;
+  if (rows > kLayoutMaxTiles) rows = kLayoutMaxTiles;
+  return (size_t)rows * (size_t)E;
+}
+
+// tables != nullptr: also add each routed token's ids into the layout tile
+// table the next place pass reads (the fused route + layout path).  `tables`
+// holds two tables of `half_words` words each.
 cudaError_t launch_route(const LaunchEnv& env, const float* logits, const float* bias, int T,
-                         int E, int k, int renorm, int32_t* ids, float* gates, WsHeader* hdr);
+                         int E, int k, int renorm, int32_t* ids, float* gates, WsHeader* hdr,
+                         uint32_t* tables = nullptr, size_t half_words = 0);
 
+// Layout of `ids` (count pass + place pass).  count_ids == false: the tile
+// table was already filled by a route launch with tables (fused path).
 cudaError_t launch_layout(const LaunchEnv& env, const int32_t* ids, int T, int E, int k, int R,
-                          int capacity, int align, int64_t N, uint32_t* status, WsHeader* hdr,
-                          int32_t* counts, int32_t* expert_off, int32_t* rank_off,
-                          int32_t* rank_counts, int32_t* dst_pos, int32_t* src_idx,
-                          uint64_t timeout_ns);
+                          int capacity, int align, int64_t N, uint32_t* tables,
+                          size_t half_words, WsHeader* hdr, int32_t* counts, int32_t* expert_off,
+                          int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
+                          int32_t* src_idx, bool count_ids = true);
 
-cudaError_t launch_route_layout(const LaunchEnv& env, const float* logits, const float* bias,
-                                int renorm, int32_t* ids, float* gates, int T, int E, int k,
-                                int R, int capacity, int align, int64_t N, uint32_t* table,
-                                WsHeader* hdr, int32_t* counts, int32_t* expert_off,
-                                int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
-                                int32_t* src_idx, uint64_t timeout_ns);
-
+// x_ready: x is not written by the kernel launched just before and every
+// earlier kernel has finished (the case right behind this library's layout
+// kernels), so x rows may be fetched before waiting on that kernel.
 cudaError_t launch_dispatch_bf16(const LaunchEnv& env, const void* x, const int32_t* dst_pos,
-                                 int T, int H, int k, int64_t N, void* out, WsHeader* hdr);
+                                 int T, int H, int k, int64_t N, void* out, WsHeader* hdr,
+                                 bool x_ready = false);
 
 cudaError_t launch_dispatch_fp8(const LaunchEnv& env, const void* x, const int32_t* dst_pos,
                                 int T, int H, int k, int64_t N, void* out, float* scales,

@@ -1,5 +1,4 @@
-// layout.cu -- steps 2 and 3: per-expert count histogram and the layout scan
-// (optionally fused with step 1, the router).
+// layout.cu -- steps 2 and 3: per-expert count histogram and the layout scan.
 //
 // "GPU MoE all-to-all" (aicassindra), section "Two collectives per layer":
 // per-destination counts precede the payload; section "Bucketing": sort rows
@@ -10,53 +9,80 @@
 // each destination's rows form one contiguous band (experts are numbered
 // rank-major, so rank slices are unions of consecutive expert segments).
 //
-// One cooperative kernel, one CTA per tile of TT tokens (all CTAs resident at
-// once, so CTAs may wait on one another; every wait is bounded):
+// Two kernels, chained by programmatic dependent launch (the kernel boundary
+// is the only grid-wide synchronisation; nothing spins):
 //
-//  1. (fused variant) route the tile's tokens, one warp per token.
-//  2. Per-warp histograms of the tile's expert ids over contiguous runs of
-//     assignments (__match_any_sync; the run leader adds), summed into the
-//     tile histogram.  No atomics, so no result depends on scheduling.
-//  3. Decoupled lookback across tiles, per expert, in an expert-major table:
-//     publish the tile's aggregate, read a window of 32 predecessors at once,
-//     add back to the nearest inclusive prefix, publish the inclusive prefix.
-//     Flag and value share one 32-bit word (flag in bits 30-31).
-//  4. The CTA of the last tile holds the totals: counts, expert offsets
-//     (segments rounded to `align`, or C rows each), rank offsets and kept
-//     rows per rank; it publishes them and raises a ready flag.
-//  5. Every CTA places its assignments: token-order rank inside the expert =
-//     tile prefix + warp prefix + lane rank within the run; capacity mode
-//     keeps ranks < C.  Writes dst_pos / src_idx and marks its share of the
-//     padding rows -1.
-//  6. Once every lookback is done, each CTA clears its table column; the last
-//     CTA to finish resets the counters, leaving the workspace ready.
+//  count  CTAs over groups of 16 tokens: shared-memory histogram of the
+//         group's expert ids, added into the row of the tile (TT consecutive
+//         tokens, about 128 tiles) the group lies in.  The fused route path
+//         does this inside the route kernel instead.
+//  place  one CTA per tile.  It sums every tile row at once (16-byte loads,
+//         one warp per row stride), so it knows each expert's total and its
+//         count in earlier tiles; a shared-memory scan over experts gives the
+//         expert offsets (segments rounded to `align`, or C rows each).  Then
+//         one pass over the tile's assignments, each warp over a contiguous
+//         run: __match_any_sync groups equal ids and the group leader advances
+//         the warp's counter, giving each assignment its rank inside the run.
+//         Token-order rank in the expert = earlier tiles + earlier warps of
+//         this tile + rank in the run.  CTA 0 writes counts and offsets.
+//
+// The tile counts live in one of two tables, alternating per call: a place
+// pass reads the table its count pass filled and clears the other one (the
+// rows the previous call left), so no clearing sits on the critical path.
+// Integer adds make every result independent of the order the CTAs run in.
 #include "common.cuh"
 #include "kernels.h"
-#include "route_core.cuh"
 
 namespace moe {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
-constexpr int kWindow = 32;
+constexpr int kCountThreads = 256;
+constexpr int kPlaceThreads = 512;
 constexpr int kUnroll = 4;
-constexpr uint32_t kFlagAgg = 1u << 30;
-constexpr uint32_t kFlagIncl = 2u << 30;
-constexpr uint32_t kValMask = (1u << 30) - 1u;
-constexpr unsigned kMaxSpins = 1u << 26;
+constexpr int kMaxStaged = 4096;  // assignments per tile kept in smem across the passes
+constexpr int kRowsInFlight = 8;  // tile rows each warp loads before adding
 
-struct LayoutParams {
-  const int32_t* ids;  // [T,k]: input, or written by step 1 in the fused kernel
-  int32_t* ids_out;    // fused: where step 1 writes the ids (same buffer)
-  const float* logits;
-  const float* bias;
-  float* gates;
-  int renorm;
-  int T, k, E, R, capacity, align, B, TT;
+__global__ void __launch_bounds__(kCountThreads)
+    count_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int TT,
+                 uint32_t* __restrict__ tables, size_t half_words, WsHeader* hdr) {
+  extern __shared__ int32_t hist[];  // [E]
+  pdl_wait();  // ids (and the tables) may come from the kernel launched before
+  pdl_trigger();
+  const uint32_t epoch = *reinterpret_cast<volatile uint32_t*>(&hdr->epoch);
+  uint32_t* tab = tables + (size_t)(epoch & 1u) * half_words;
+  for (int e = threadIdx.x; e < E; e += kCountThreads) hist[e] = 0;
+  __syncthreads();
+  for (int g0 = blockIdx.x * kLayoutTileQuantum; g0 < T; g0 += gridDim.x * kLayoutTileQuantum) {
+    const int64_t i0 = (int64_t)g0 * k;
+    const int64_t i1 = (int64_t)min(T, g0 + kLayoutTileQuantum) * k;
+    for (int64_t i = i0 + threadIdx.x; i < i1; i += kCountThreads) {
+      const int e = __ldg(ids + i);
+      if ((unsigned)e < (unsigned)E)
+        atomicAdd(&hist[e], 1);
+      else
+        report(hdr, MOE_ERR_DEVICE_RANGE, (int)i);
+    }
+    __syncthreads();
+    uint32_t* row = tab + (size_t)(g0 / TT) * E;  // the group lies in one tile
+    for (int e = threadIdx.x; e < E; e += kCountThreads) {
+      const int c = hist[e];
+      if (c != 0) {
+        atomicAdd(row + e, (uint32_t)c);
+        hist[e] = 0;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+struct PlaceParams {
+  const int32_t* ids;
+  int T, k, E, R, capacity, align, G, TT;
+  int staged;
   int64_t N;
-  uint32_t* table;  // [E][B] lookback words
+  uint32_t* tables;
+  size_t half_words;
   WsHeader* hdr;
   int32_t* counts;
   int32_t* expert_off;
@@ -64,71 +90,15 @@ struct LayoutParams {
   int32_t* rank_counts;
   int32_t* dst_pos;
   int32_t* src_idx;
-  uint64_t timeout_ns;
 };
 
-// Wait until the word at p carries a flag; after the time limit record
-// MOE_ERR_DEVICE_TIMEOUT and return a placeholder inclusive 0.
-__device__ __noinline__ uint32_t wait_word(const uint32_t* p, WsHeader* hdr, uint64_t timeout_ns,
-                                           int who) {
-  const uint64_t t0 = global_ns();
-  for (unsigned it = 0; it < kMaxSpins; ++it) {
-    const uint32_t w = ld_relaxed(p);
-    if (w & ~kValMask) return w;
-    if ((it & 15u) == 15u) {
-      if (error_seen(hdr) == MOE_ERR_DEVICE_TIMEOUT) return kFlagIncl;
-      if (global_ns() - t0 > timeout_ns) break;
-    }
-    __nanosleep(64);
-  }
-  report(hdr, MOE_ERR_DEVICE_TIMEOUT, who);
-  return kFlagIncl;
-}
-
-// Wait until *p >= target; false (and MOE_ERR_DEVICE_TIMEOUT) after the limit.
-__device__ __noinline__ bool wait_count(const uint32_t* p, uint32_t target, WsHeader* hdr,
-                                        uint64_t timeout_ns, int who) {
-  const uint64_t t0 = global_ns();
-  for (unsigned it = 0; it < kMaxSpins; ++it) {
-    if (ld_acquire(p) >= target) return true;
-    if ((it & 15u) == 15u) {
-      if (error_seen(hdr) == MOE_ERR_DEVICE_TIMEOUT) return false;
-      if (global_ns() - t0 > timeout_ns) break;
-    }
-    __nanosleep(128);
-  }
-  report(hdr, MOE_ERR_DEVICE_TIMEOUT, who);
-  return false;
-}
-
-// Exclusive prefix of tile vb for one expert: sum the predecessors' words from
-// the nearest back to the first inclusive one, 32 loads in flight at a time.
-__device__ uint32_t lookback(const uint32_t* col, int vb, WsHeader* hdr, uint64_t timeout_ns) {
-  uint32_t excl = 0;
-  for (int hi = vb - 1; hi >= 0; hi -= kWindow) {
-    uint32_t w[kWindow];
-#pragma unroll
-    for (int i = 0; i < kWindow; ++i) w[i] = (hi - i >= 0) ? ld_relaxed(col + hi - i) : 0u;
-    bool done = false;
-#pragma unroll
-    for (int i = 0; i < kWindow; ++i) {
-      if (!done && hi - i >= 0) {
-        uint32_t v = w[i];
-        if ((v & ~kValMask) == 0u) v = wait_word(col + hi - i, hdr, timeout_ns, vb);
-        excl += v & kValMask;
-        done = (v & ~kValMask) == kFlagIncl;
-      }
-    }
-    if (done) break;
-  }
-  return excl & kValMask;
-}
-
 // Exclusive scan of v[0..n) in shared memory by the whole CTA (n <= 4 *
-// kThreads).  Returns the total to every thread.
+// THREADS).  Returns the total to every thread.
+template <int THREADS>
 __device__ int block_exclusive_scan(int32_t* v, int n, int32_t* warp_tot) {
+  constexpr int kW = THREADS / 32;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int per = (n + kThreads - 1) / kThreads;
+  const int per = (n + THREADS - 1) / THREADS;
   const int lo = threadIdx.x * per;
   int local = 0;
   for (int i = 0; i < per; ++i)
@@ -142,17 +112,17 @@ __device__ int block_exclusive_scan(int32_t* v, int n, int32_t* warp_tot) {
   if (lane == 31) warp_tot[wid] = x;
   __syncthreads();
   if (wid == 0) {
-    int s = (lane < kWarps) ? warp_tot[lane] : 0;
+    int s = (lane < kW) ? warp_tot[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(kFull, s, o);
       if (lane >= o) s += y;
     }
-    if (lane < kWarps) warp_tot[lane] = s;
+    if (lane < kW) warp_tot[lane] = s;
   }
   __syncthreads();
   int run = (wid > 0 ? warp_tot[wid - 1] : 0) + x - local;
-  const int total = warp_tot[kWarps - 1];
+  const int total = warp_tot[kW - 1];
   for (int i = 0; i < per; ++i)
     if (lo + i < n) {
       const int t = v[lo + i];
@@ -163,184 +133,215 @@ __device__ int block_exclusive_scan(int32_t* v, int n, int32_t* warp_tot) {
   return total;
 }
 
-template <int NK, bool ROUTE>
-__global__ void __launch_bounds__(kThreads) layout_kernel(const LayoutParams P) {
+constexpr size_t place_smem_words(int E, int staged_entries) {
+  return (size_t)(kPlaceThreads / 32) * E + 4 * (size_t)E + 1 + 2 * (size_t)staged_entries;
+}
+
+__global__ void __launch_bounds__(kPlaceThreads) place_kernel(const PlaceParams P) {
+  constexpr int kW = kPlaceThreads / 32;
   extern __shared__ int32_t smem[];
   const int E = P.E, k = P.k, C = P.capacity;
-  int32_t* wh = smem;                // [kWarps][E] per-warp counts, then bases
-  int32_t* tile = wh + kWarps * E;   // [E] tile histogram, then inclusive prefix
-  int32_t* off = tile + E;           // [E+1] expert offsets
-  int32_t* kept = off + E + 1;       // [E]
-  __shared__ int32_t s_wtot[kWarps];
+  int32_t* wh = smem;             // [kW][E] per-warp counts, then tile-local warp bases
+  int32_t* pre = wh + kW * E;     // [E] count in earlier tiles
+  int32_t* tot = pre + E;         // [E] total count
+  int32_t* off = tot + E;         // [E+1] expert offsets
+  int32_t* kept = off + E + 1;    // [E] rows kept per expert
+  int32_t* sid = kept + E;        // [TT*k] staged expert ids
+  int32_t* srk = sid + P.TT * k;  // [TT*k] staged ranks inside the warp's run
+  __shared__ int32_t s_wtot[kW];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int vb = blockIdx.x;
   const int t0 = min(P.T, vb * P.TT);
   const int t1 = min(P.T, t0 + P.TT);
-
-  if constexpr (ROUTE) {
-    float b[NK];
-    load_bias<NK>(P.bias, E, lane, b);
-    for (int t = t0 + w; t < t1; t += kWarps) {
-      int e;
-      float g;
-      bool nan_key;
-      route_token<NK>(P.logits + (size_t)t * E, b, E, k, P.renorm, lane, e, g, nan_key);
-      if (nan_key && lane == 0) report(P.hdr, MOE_ERR_DEVICE_NAN, t);
-      if (lane < k) {
-        P.ids_out[(size_t)t * k + lane] = e;
-        P.gates[(size_t)t * k + lane] = g;
-      }
-    }
-  }
-  for (int i = threadIdx.x; i < kWarps * E; i += kThreads) wh[i] = 0;
-  __syncthreads();  // (fused) the tile's ids are written before anyone reads them
-
-  // this warp's contiguous run of the tile's assignments
   const int64_t i0 = (int64_t)t0 * k, i1 = (int64_t)t1 * k;
-  const int64_t chunk = (((i1 - i0) + kWarps - 1) / kWarps + 31) / 32 * 32;
+
+  pdl_wait();  // the count pass has finished
+  pdl_trigger();
+  // epoch, done, words_used[0..1] in one load
+  const uint4 hv = __ldcg(reinterpret_cast<const uint4*>(&P.hdr->epoch));
+  const uint32_t epoch = hv.x;
+  const uint32_t cur_b = epoch & 1u, oth_b = cur_b ^ 1u;
+  const uint32_t* cur = P.tables + (size_t)cur_b * P.half_words;
+  uint32_t* oth = P.tables + (size_t)oth_b * P.half_words;
+  const uint32_t oth_used = oth_b ? hv.w : hv.z;
+  for (int i = threadIdx.x; i < kW * E; i += kPlaceThreads) wh[i] = 0;
+  for (int e = threadIdx.x; e < E; e += kPlaceThreads) {
+    pre[e] = 0;
+    tot[e] = 0;
+  }
+  // this warp's contiguous run of the tile's assignments; its first ids are
+  // fetched now so their latency overlaps the table reads below
+  const int64_t chunk = (((i1 - i0) + kW - 1) / kW + 31) / 32 * 32;
   const int64_t s0 = min(i1, i0 + (int64_t)w * chunk);
   const int64_t s1 = min(i1, s0 + chunk);
-  int32_t* my = wh + w * E;
+  int ev0[kUnroll];
+#pragma unroll
+  for (int u = 0; u < kUnroll; ++u) {
+    const int64_t i = s0 + 32 * u + lane;
+    ev0[u] = (i < s1) ? __ldg(P.ids + i) : -1;
+  }
+  __syncthreads();
 
-  // pass 1: per-warp histogram
-  for (int64_t base = s0; base < s1; base += 32 * kUnroll) {
-    int ev[kUnroll];
+  // 1. every tile row: totals and the count in earlier tiles
+  if ((E & 3) == 0) {
+    for (int eb = 4 * lane; eb < E; eb += 128) {
+      uint4 at = make_uint4(0, 0, 0, 0), ap = make_uint4(0, 0, 0, 0);
+      for (int p0 = w; p0 < P.G; p0 += kW * kRowsInFlight) {
+        uint4 v[kRowsInFlight];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t i = base + 32 * u + lane;
-      ev[u] = (i < s1) ? P.ids[i] : -1;
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t i = base + 32 * u + lane;
-      if (base + 32 * u < s1) {
-        const bool ok = (i < s1) && (unsigned)ev[u] < (unsigned)E;
-        if (i < s1 && !ok) report(P.hdr, MOE_ERR_DEVICE_RANGE, (int)i);
-        const unsigned active = __ballot_sync(kFull, ok);
-        if (ok) {
-          const unsigned peers = __match_any_sync(active, ev[u]);
-          if (lane == __ffs(peers) - 1) my[ev[u]] += __popc(peers);
+        for (int r = 0; r < kRowsInFlight; ++r) {
+          const int p = p0 + r * kW;
+          v[r] = (p < P.G) ? __ldcg(reinterpret_cast<const uint4*>(cur + (size_t)p * E + eb))
+                           : make_uint4(0, 0, 0, 0);
         }
-        __syncwarp();
+#pragma unroll
+        for (int r = 0; r < kRowsInFlight; ++r) {
+          at.x += v[r].x;
+          at.y += v[r].y;
+          at.z += v[r].z;
+          at.w += v[r].w;
+          if (p0 + r * kW < vb) {
+            ap.x += v[r].x;
+            ap.y += v[r].y;
+            ap.z += v[r].z;
+            ap.w += v[r].w;
+          }
+        }
       }
+      atomicAdd(&tot[eb + 0], (int)at.x);
+      atomicAdd(&tot[eb + 1], (int)at.y);
+      atomicAdd(&tot[eb + 2], (int)at.z);
+      atomicAdd(&tot[eb + 3], (int)at.w);
+      atomicAdd(&pre[eb + 0], (int)ap.x);
+      atomicAdd(&pre[eb + 1], (int)ap.y);
+      atomicAdd(&pre[eb + 2], (int)ap.z);
+      atomicAdd(&pre[eb + 3], (int)ap.w);
+    }
+  } else {
+    for (int e = lane; e < E; e += 32) {
+      int at = 0, ap = 0;
+      for (int p = w; p < P.G; p += kW) {
+        const int v = (int)__ldcg(cur + (size_t)p * E + e);
+        at += v;
+        if (p < vb) ap += v;
+      }
+      atomicAdd(&tot[e], at);
+      atomicAdd(&pre[e], ap);
     }
   }
   __syncthreads();
 
-  // tile histogram; publish the aggregate (tile 0: its inclusive prefix)
-  for (int e = threadIdx.x; e < E; e += kThreads) {
-    int h = 0;
-    for (int q = 0; q < kWarps; ++q) h += wh[q * E + e];
-    tile[e] = h;
-    st_relaxed(P.table + (size_t)e * P.B + vb, (vb == 0 ? kFlagIncl : kFlagAgg) | (uint32_t)h);
-  }
-  // lookback; then each warp's first token-order rank in each expert
-  for (int e = threadIdx.x; e < E; e += kThreads) {
-    const uint32_t ex = (vb > 0) ? lookback(P.table + (size_t)e * P.B, vb, P.hdr, P.timeout_ns)
-                                 : 0u;
-    if (vb > 0)
-      st_relaxed(P.table + (size_t)e * P.B + vb, kFlagIncl | ((ex + (uint32_t)tile[e]) & kValMask));
-    int run = (int)ex;
-    for (int q = 0; q < kWarps; ++q) {
-      const int c = wh[q * E + e];
-      wh[q * E + e] = run;
-      run += c;
-    }
-    tile[e] = run;
+  // 2. expert offsets (every CTA computes the same scan); CTA 0 publishes them
+  for (int e = threadIdx.x; e < E; e += kPlaceThreads) {
+    const int c = tot[e];
+    off[e] = C > 0 ? C : ((c + P.align - 1) / P.align) * P.align;
+    kept[e] = (C > 0 && c > C) ? C : c;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(&P.hdr->looked, 1u);
-  }
-
-  // the last tile's inclusive prefixes are the totals
-  if (vb == P.B - 1) {
-    for (int e = threadIdx.x; e < E; e += kThreads) {
-      const int c = tile[e];
-      P.counts[e] = c;
-      off[e] = C > 0 ? C : ((c + P.align - 1) / P.align) * P.align;
-      kept[e] = (C > 0 && c > C) ? C : c;
-    }
-    __syncthreads();
-    const int used = block_exclusive_scan(off, E, s_wtot);
-    const int kept_total = block_exclusive_scan(kept, E, s_wtot);
+  const int used = block_exclusive_scan<kPlaceThreads>(off, E, s_wtot);
+  if (threadIdx.x == 0) off[E] = used;
+  if (vb == 0) {
     const int Er = E / P.R;
-    for (int e = threadIdx.x; e < E; e += kThreads) P.expert_off[e] = off[e];
-    for (int r = threadIdx.x; r < P.R; r += kThreads) {
-      P.rank_off[r] = off[r * Er];
-      const int hi = (r + 1 < P.R) ? kept[(r + 1) * Er] : kept_total;
-      P.rank_counts[r] = hi - kept[r * Er];
+    for (int e = threadIdx.x; e < E; e += kPlaceThreads) {
+      P.counts[e] = tot[e];
+      P.expert_off[e] = off[e];
+    }
+    for (int r = w; r < P.R; r += kW) {  // one warp per rank: rows kept
+      int s = 0;
+      for (int e = r * Er + lane; e < (r + 1) * Er; e += 32) s += kept[e];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(kFull, s, o);
+      if (lane == 0) {
+        P.rank_counts[r] = s;
+        P.rank_off[r] = off[r * Er];
+      }
     }
     if (threadIdx.x == 0) {
       P.expert_off[E] = used;
       P.rank_off[P.R] = used;
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      __threadfence();
-      st_release(&P.hdr->totals_ready, 1u);
-    }
   }
-  if (threadIdx.x == 0) wait_count(&P.hdr->totals_ready, 1u, P.hdr, P.timeout_ns, vb);
-  __syncthreads();
-  const bool fill = (C > 0 || P.align > 1);
-  for (int e = threadIdx.x; e <= E; e += kThreads) off[e] = ld_cg(P.expert_off + e);
-  if (fill)
-    for (int e = threadIdx.x; e < E; e += kThreads) {
-      const int c = ld_cg(P.counts + e);
-      kept[e] = (C > 0 && c > C) ? C : c;
-    }
-  __syncthreads();
 
-  // pass 2: place each assignment at its token-order rank
-  for (int64_t base = s0; base < s1; base += 32 * kUnroll) {
-    int ev[kUnroll];
+  // 3. this tile's assignments: per-warp counts and each one's rank in its run
+  int32_t* my = wh + w * E;
+  auto run_ranks = [&](auto&& emit, bool first_prefetched) {
+    for (int64_t base = s0; base < s1; base += 32 * kUnroll) {
+      int ev[kUnroll];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t i = base + 32 * u + lane;
-      ev[u] = (i < s1) ? P.ids[i] : -1;
-    }
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t i = base + 32 * u + lane;
+        ev[u] = (first_prefetched && base == s0) ? ev0[u] : ((i < s1) ? __ldg(P.ids + i) : -1);
+      }
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t i = base + 32 * u + lane;
-      if (base + 32 * u < s1) {
-        const int e = ev[u];
-        const bool ok = (i < s1) && (unsigned)e < (unsigned)E;
-        const unsigned active = __ballot_sync(kFull, ok);
-        int v = 0, cnt = 0;
-        bool lead = false;
-        if (ok) {
-          const unsigned peers = __match_any_sync(active, e);
-          v = my[e] + __popc(peers & lanemask_lt());
-          lead = (lane == __ffs(peers) - 1);
-          cnt = __popc(peers);
-        }
-        __syncwarp();
-        if (lead) my[e] = v + cnt;
-        __syncwarp();
-        if (i < s1) {
-          int64_t dst = -1;
-          if (ok) dst = (C > 0) ? (v < C ? (int64_t)e * C + v : -1) : (int64_t)off[e] + v;
-          // in range by construction; checked because a lookback that gave up
-          // leaves placeholder prefixes
-          if (dst >= P.N || (ok && v < 0)) {
-            report(P.hdr, MOE_ERR_DEVICE_RANGE, (int)dst);
-            dst = -1;
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t i = base + 32 * u + lane;
+        if (base + 32 * u < s1) {
+          const int e = ev[u];
+          const bool ok = (i < s1) && (unsigned)e < (unsigned)E;
+          const unsigned active = __ballot_sync(kFull, ok);
+          int v = -1;
+          if (ok) {
+            const unsigned peers = __match_any_sync(active, e);
+            v = my[e] + __popc(peers & lanemask_lt());
+            __syncwarp(active);
+            if (lane == __ffs(peers) - 1) my[e] = v + __popc(peers);
           }
-          P.dst_pos[i] = (int32_t)dst;
-          if (dst >= 0) P.src_idx[dst] = (int32_t)i;
+          __syncwarp();
+          if (i < s1) emit(i, e, v);
         }
       }
     }
+  };
+  if (P.staged)
+    run_ranks(
+        [&](int64_t i, int e, int v) {
+          sid[i - i0] = e;
+          srk[i - i0] = v;
+        },
+        true);
+  else
+    run_ranks([](int64_t, int, int) {}, true);
+  __syncthreads();
+  // per-warp counts -> tile-local bases (warps in token order)
+  for (int e = threadIdx.x; e < E; e += kPlaceThreads) {
+    int run = pre[e];
+    for (int q = 0; q < kW; ++q) {
+      const int c = wh[q * E + e];
+      wh[q * E + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+
+  // 4. place each assignment at its row
+  auto place = [&](int64_t i, int e, int rank) {
+    int64_t dst = -1;
+    if (rank >= 0)
+      dst = (C > 0) ? (rank < C ? (int64_t)e * C + rank : -1) : (int64_t)off[e] + rank;
+    if (dst >= P.N) {  // in range by construction; guards a corrupted tile table
+      report(P.hdr, MOE_ERR_DEVICE_RANGE, (int)(dst > INT32_MAX ? INT32_MAX : dst));
+      dst = -1;
+    }
+    P.dst_pos[i] = (int32_t)dst;
+    if (dst >= 0) P.src_idx[dst] = (int32_t)i;
+  };
+  if (P.staged) {
+    for (int64_t r = threadIdx.x; r < i1 - i0; r += kPlaceThreads) {
+      const int e = sid[r];
+      const int v = srk[r];
+      const int q = (int)(r / chunk);  // the warp whose run holds r
+      place(i0 + r, e, v < 0 ? -1 : wh[q * E + e] + v);
+    }
+  } else {
+    run_ranks([&](int64_t i, int e, int v) { place(i, e, v); }, true);  // my[] starts at the bases
   }
 
-  // rows that hold no assignment (alignment padding, unused capacity slots)
-  if (fill) {
-    const int64_t per = (P.N + P.B - 1) / P.B;
+  // 5. rows that hold no assignment (alignment padding, unused capacity slots)
+  if (C > 0 || P.align > 1) {
+    const int64_t per = (P.N + P.G - 1) / P.G;
     const int64_t r0 = (int64_t)vb * per;
     const int64_t r1 = min(P.N, r0 + per);
-    for (int64_t p = r0 + threadIdx.x; p < r1; p += kThreads) {
+    for (int64_t p = r0 + threadIdx.x; p < r1; p += kPlaceThreads) {
       bool pad = true;
       if (p < off[E]) {
         int lo = 0, hi = E - 1;  // last e with off[e] <= p
@@ -357,60 +358,47 @@ __global__ void __launch_bounds__(kThreads) layout_kernel(const LayoutParams P) 
     }
   }
 
-  // once no lookback reads the table any more, clear this tile's column
-  if (threadIdx.x == 0) wait_count(&P.hdr->looked, (uint32_t)P.B, P.hdr, P.timeout_ns, vb);
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += kThreads) P.table[(size_t)e * P.B + vb] = 0u;
+  // 6. clear what the previous call left in the other table; the last CTA to
+  //    finish flips the tables for the next call
+  for (size_t x = (size_t)vb * kPlaceThreads + threadIdx.x; x < oth_used;
+       x += (size_t)P.G * kPlaceThreads)
+    oth[x] = 0u;
+  // (everything here is read only by the next call, after this kernel has
+  // completed, so the counter needs no fence)
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
-    if (atomicAdd(&P.hdr->finished, 1u) == (uint32_t)P.B - 1u) {
-      P.hdr->looked = 0u;
-      P.hdr->totals_ready = 0u;
-      P.hdr->finished = 0u;
+    if (atomicAdd(&P.hdr->done, 1u) == (uint32_t)P.G - 1u) {
+      P.hdr->words_used[cur_b] = (uint32_t)((size_t)P.G * E);
+      P.hdr->words_used[oth_b] = 0u;
+      P.hdr->done = 0u;
+      P.hdr->epoch = epoch + 1u;
     }
   }
-}
-
-template <int NK, bool ROUTE>
-cudaError_t launch_fused(const LaunchEnv& env, LayoutParams P) {
-  auto kern = layout_kernel<NK, ROUTE>;
-  const size_t smem = (11 * (size_t)P.E + 1) * sizeof(int32_t);
-  int per_sm = 0;
-  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
-  if (err != cudaSuccess) return err;
-  if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  const int64_t max_blocks = (int64_t)per_sm * env.num_sms;
-  // tiles of 128 tokens, doubled until every tile's CTA can be resident at once
-  int64_t TT = kLayoutTileTokens;
-  int64_t B = P.T > 0 ? (P.T + TT - 1) / TT : 1;
-  while (B > max_blocks) {
-    TT *= 2;
-    B = (P.T + TT - 1) / TT;
-  }
-  P.TT = (int)TT;
-  P.B = (int)B;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)B);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = env.stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, P);
 }
 
 }  // namespace
 
 cudaError_t launch_layout(const LaunchEnv& env, const int32_t* ids, int T, int E, int k, int R,
-                          int capacity, int align, int64_t N, uint32_t* table, WsHeader* hdr,
-                          int32_t* counts, int32_t* expert_off, int32_t* rank_off,
-                          int32_t* rank_counts, int32_t* dst_pos, int32_t* src_idx,
-                          uint64_t timeout_ns) {
-  LayoutParams P{};
+                          int capacity, int align, int64_t N, uint32_t* tables,
+                          size_t half_words, WsHeader* hdr, int32_t* counts, int32_t* expert_off,
+                          int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
+                          int32_t* src_idx, bool count_ids) {
+  const TileGeom geom = layout_tiles(T);
+  cudaError_t err;
+  if (count_ids && T > 0) {
+    const size_t smem = (size_t)E * sizeof(int32_t);
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, count_kernel, kCountThreads, smem);
+    if (err != cudaSuccess) return err;
+    if (per_sm < 1) per_sm = 1;
+    int64_t blocks = ((int64_t)T + kLayoutTileQuantum - 1) / kLayoutTileQuantum;
+    const int64_t cap = (int64_t)per_sm * env.num_sms;
+    if (blocks > cap) blocks = cap;
+    err = launch_pdl(env, count_kernel, dim3((unsigned)blocks), dim3(kCountThreads), smem, ids, T,
+                     k, E, geom.TT, tables, half_words, hdr);
+    if (err != cudaSuccess) return err;
+  }
+  PlaceParams P{};
   P.ids = ids;
   P.T = T;
   P.k = k;
@@ -418,8 +406,11 @@ cudaError_t launch_layout(const LaunchEnv& env, const int32_t* ids, int T, int E
   P.R = R;
   P.capacity = capacity;
   P.align = align;
+  P.G = geom.G;
+  P.TT = geom.TT;
   P.N = N;
-  P.table = table;
+  P.tables = tables;
+  P.half_words = half_words;
   P.hdr = hdr;
   P.counts = counts;
   P.expert_off = expert_off;
@@ -427,46 +418,15 @@ cudaError_t launch_layout(const LaunchEnv& env, const int32_t* ids, int T, int E
   P.rank_counts = rank_counts;
   P.dst_pos = dst_pos;
   P.src_idx = src_idx;
-  P.timeout_ns = timeout_ns;
-  return launch_fused<1, false>(env, P);
-}
-
-cudaError_t launch_route_layout(const LaunchEnv& env, const float* logits, const float* bias,
-                                int renorm, int32_t* ids, float* gates, int T, int E, int k,
-                                int R, int capacity, int align, int64_t N, uint32_t* table,
-                                WsHeader* hdr, int32_t* counts, int32_t* expert_off,
-                                int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
-                                int32_t* src_idx, uint64_t timeout_ns) {
-  LayoutParams P{};
-  P.ids = ids;
-  P.ids_out = ids;
-  P.logits = logits;
-  P.bias = bias;
-  P.gates = gates;
-  P.renorm = renorm;
-  P.T = T;
-  P.k = k;
-  P.E = E;
-  P.R = R;
-  P.capacity = capacity;
-  P.align = align;
-  P.N = N;
-  P.table = table;
-  P.hdr = hdr;
-  P.counts = counts;
-  P.expert_off = expert_off;
-  P.rank_off = rank_off;
-  P.rank_counts = rank_counts;
-  P.dst_pos = dst_pos;
-  P.src_idx = src_idx;
-  P.timeout_ns = timeout_ns;
-  const int nk = (E + 31) / 32;
-  if (nk <= 1) return launch_fused<1, true>(env, P);
-  if (nk <= 2) return launch_fused<2, true>(env, P);
-  if (nk <= 4) return launch_fused<4, true>(env, P);
-  if (nk <= 8) return launch_fused<8, true>(env, P);
-  if (nk <= 16) return launch_fused<16, true>(env, P);
-  return launch_fused<32, true>(env, P);
+  const int64_t entries = (int64_t)geom.TT * k;
+  P.staged = entries <= kMaxStaged ? 1 : 0;
+  const size_t smem = place_smem_words(E, P.staged ? (int)entries : 0) * sizeof(int32_t);
+  if (smem > 48 * 1024) {
+    err = cudaFuncSetAttribute(place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+    if (err != cudaSuccess) return err;
+  }
+  return launch_pdl(env, place_kernel, dim3((unsigned)geom.G), dim3(kPlaceThreads), smem, P);
 }
 
 }  // namespace moe

@@ -6,15 +6,16 @@
 // runtimes whose memory pool owns every byte of the device, and code on a
 // latency-critical path where cudaMalloc (which may synchronise the device)
 // is not allowed.  This entry point runs the same count and place kernels as
-// moe_layout, with their scratch (error word, block ticket and the per-tile
-// prefix table) in a file-scope device array instead of a caller workspace.
+// moe_layout, with their scratch (error word, the layout's counters and its
+// two tile tables) in a file-scope device array instead of a caller workspace.
 //
 // The array is kMoeNoallocScratchBytes bytes; every GPU that loads the library
 // holds it until the process exits.  The first call on a device looks up its
 // device address (cudaGetSymbolAddress, with that device current) and clears
-// it; make that first call before any stream capture.  Each call then clears
-// the header (error word and ticket) on the caller's stream.  Calls share the
-// array, so calls that overlap on the GPU (different streams, or different
+// it; make that first call before any stream capture.  Every call leaves the
+// array ready for the next one (the layout kernels clear the counters they
+// used); a call whose launch fails clears the whole array again.  Calls share
+// the array, so calls that overlap on the GPU (different streams, or different
 // host threads, without ordering) race and give wrong results.
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -81,8 +82,6 @@ extern "C" moe_status_t moe_layout_noalloc(const moe_shape_t* shape, const int32
   void* scratch = nullptr;
   moe_status_t st = scratch_for_current_device(s, &scratch);
   if (st != MOE_OK) return st;
-  // error word and ticket start at zero for every call
-  if (cudaMemsetAsync(scratch, 0, kHeader, s) != cudaSuccess) return MOE_ERR_CUDA;
 
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
@@ -92,10 +91,15 @@ extern "C" moe_status_t moe_layout_noalloc(const moe_shape_t* shape, const int32
   env.stream = s;
   env.num_sms = sms;
   moe::WsHeader* hdr = static_cast<moe::WsHeader*>(scratch);
-  uint32_t* table = reinterpret_cast<uint32_t*>(static_cast<char*>(scratch) + kHeader);
+  uint32_t* tables = reinterpret_cast<uint32_t*>(static_cast<char*>(scratch) + kHeader);
+  const size_t half_words = (MOE_NOALLOC_TABLE_BYTES / 8) / 4 * 4;
   const cudaError_t err = moe::launch_layout(
       env, ids, shape->tokens, shape->experts, shape->k, shape->ranks, shape->capacity,
-      shape->align, rows, table, hdr, counts, expert_off, rank_off, rank_counts, dst_pos,
-      src_idx, 1000000000ull);
-  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+      shape->align, rows, tables, half_words, hdr, counts, expert_off, rank_off, rank_counts,
+      dst_pos, src_idx, true);
+  if (err != cudaSuccess) {
+    (void)cudaMemsetAsync(scratch, 0, kMoeNoallocScratchBytes, s);  // back to a clean array
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
 }

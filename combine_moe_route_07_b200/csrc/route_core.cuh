@@ -1,17 +1,18 @@
-// route_core.cuh -- one token's top-k selection and gates, executed by one
-// warp.  Shared by the standalone route kernel and the fused route + layout
-// kernel.
+// route_core.cuh -- top-k selection and gates for a few tokens at once, one
+// warp per group.  Shared by the standalone route kernel and the fused
+// route + layout kernel.
 //
 // "19. All-to-all" (ai-from-scratch), section "Why the router can ruin your
 // day": the per-expert balancing bias enters the top-k decision and nothing
 // else; the mix weights come from the router's own scores.
 //
-// Lane l holds experts l, l+32, l+64, ... in registers as order-preserving
-// 32-bit codes of key = logit + bias.  Each of the k rounds is two hardware
-// warp reductions (redux.sync): the largest code, then the lowest expert id
-// among the lanes holding it, which is the tie rule.  The gates are a softmax
-// of the selected RAW logits evaluated in fp64 (k values per token, off the
-// memory-bound path) and rounded to fp32 once.
+// Lane l holds experts l, l+32, l+64, ... of each token in registers, as
+// order-preserving 32-bit codes of key = logit + bias.  Each of the k rounds
+// is two hardware warp reductions (redux.sync): the largest code, then the
+// lowest expert id among the lanes holding it, which is the tie rule.  TPW
+// tokens go through the rounds together so their latency chains overlap.
+// The gates are a softmax of the selected RAW logits evaluated in fp64 (k
+// values per token) and rounded to fp32 once.
 #pragma once
 
 #include <math.h>
@@ -49,76 +50,99 @@ __device__ __forceinline__ void load_bias(const float* bias, int E, int lane, fl
   }
 }
 
-// Route the token whose logits start at `row`.  On return lane j < k holds
-// slot j: expert `sel_e` and gate `gate`.  `nan_key` is set on every lane if
-// any key of the token was NaN.
+// Tokens per warp group for NK keys per lane (register budget).
 template <int NK>
-__device__ __forceinline__ void route_token(const float* __restrict__ row, const float (&b)[NK],
-                                            int E, int k, int renorm, int lane, int& sel_e,
-                                            float& gate, bool& nan_key) {
-  float raw[NK];
-  uint32_t code[NK];
-  bool bad = false;
-#pragma unroll
-  for (int i = 0; i < NK; ++i) {
-    const int e = lane + 32 * i;
-    if (e < E) {
-      raw[i] = __ldcs(row + e);  // read once: streaming
-      const float key = __fadd_rn(raw[i], b[i]);
-      bad |= (key != key);
-      code[i] = order_code(key);
-    } else {
-      raw[i] = -INFINITY;
-      code[i] = 0u;
-    }
-  }
-  nan_key = __any_sync(kFull, bad);
+struct RouteGroup {
+  static constexpr int value = NK <= 4 ? 4 : (NK <= 8 ? 2 : 1);
+};
 
-  sel_e = 0;
-  float sel_raw = 0.0f;
+// Route tokens tok[0..TPW) (entries >= T are skipped).  On return lane j < k
+// holds slot j of token u: expert sel_e[u], gate[u].  Returns the first token
+// with a NaN key, or -1.
+template <int NK, int TPW>
+__device__ __forceinline__ int route_tokens(const float* __restrict__ logits, const int (&tok)[TPW],
+                                            int T, const float (&b)[NK], int E, int k, int renorm,
+                                            int lane, int (&sel_e)[TPW], float (&gate)[TPW]) {
+  float raw[TPW][NK];
+  uint32_t code[TPW][NK];
+  int nan_tok = -1;
+#pragma unroll
+  for (int u = 0; u < TPW; ++u) {
+    const bool live = tok[u] < T;
+    const float* row = logits + (size_t)(live ? tok[u] : 0) * E;
+    bool bad = false;
+#pragma unroll
+    for (int i = 0; i < NK; ++i) {
+      const int e = lane + 32 * i;
+      if (live && e < E) {
+        raw[u][i] = __ldcs(row + e);  // read once: streaming
+        const float key = __fadd_rn(raw[u][i], b[i]);
+        bad |= (key != key);
+        code[u][i] = order_code(key);
+      } else {
+        raw[u][i] = -INFINITY;
+        code[u][i] = 0u;
+      }
+    }
+    if (__any_sync(kFull, bad) && nan_tok < 0) nan_tok = tok[u];
+  }
+
+  float sel_raw[TPW];
+#pragma unroll
+  for (int u = 0; u < TPW; ++u) {
+    sel_e[u] = 0;
+    sel_raw[u] = 0.0f;
+  }
   for (int j = 0; j < k; ++j) {
-    uint32_t best = 0u;
-    int bi = 0;
 #pragma unroll
-    for (int i = 0; i < NK; ++i)
-      if (code[i] > best) {  // strict: the lowest index wins ties
-        best = code[i];
-        bi = i;
-      }
-    const uint32_t top = __reduce_max_sync(kFull, best);
-    const uint32_t cand = (best == top) ? (uint32_t)(lane + 32 * bi) : 0xffffffffu;
-    const uint32_t win = __reduce_min_sync(kFull, cand);
-    float r = 0.0f;
+    for (int u = 0; u < TPW; ++u) {
+      uint32_t best = 0u;
+      int bi = 0;
 #pragma unroll
-    for (int i = 0; i < NK; ++i)
-      if ((uint32_t)(lane + 32 * i) == win) {
-        code[i] = 0u;
-        r = raw[i];
+      for (int i = 0; i < NK; ++i)
+        if (code[u][i] > best) {  // strict: the lowest index wins ties
+          best = code[u][i];
+          bi = i;
+        }
+      const uint32_t top = __reduce_max_sync(kFull, best);
+      const uint32_t cand = (best == top) ? (uint32_t)(lane + 32 * bi) : 0xffffffffu;
+      const uint32_t win = __reduce_min_sync(kFull, cand);
+      float r = 0.0f;
+#pragma unroll
+      for (int i = 0; i < NK; ++i)
+        if ((uint32_t)(lane + 32 * i) == win) {
+          code[u][i] = 0u;
+          r = raw[u][i];
+        }
+      r = __shfl_sync(kFull, r, (int)(win & 31u));
+      if (lane == j) {
+        sel_e[u] = (int)win;
+        sel_raw[u] = r;
       }
-    r = __shfl_sync(kFull, r, (int)(win & 31u));
-    if (lane == j) {
-      sel_e = (int)win;
-      sel_raw = r;
     }
   }
 
-  if (renorm) {
-    const float m = warp_max_f(lane < k ? sel_raw : -INFINITY);
-    const double ex = (lane < k) ? exp((double)sel_raw - (double)m) : 0.0;
-    const double den = warp_sum_d(ex);
-    gate = (float)(ex / den);
-  } else {
-    float lm = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < NK; ++i) lm = fmaxf(lm, raw[i]);
-    const float m = warp_max_f(lm);
-    double part = 0.0;
+  for (int u = 0; u < TPW; ++u) {
+    if (renorm) {
+      const float m = warp_max_f(lane < k ? sel_raw[u] : -INFINITY);
+      const double ex = (lane < k) ? exp((double)sel_raw[u] - (double)m) : 0.0;
+      const double den = warp_sum_d(ex);
+      gate[u] = (float)(ex / den);
+    } else {
+      float lm = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < NK; ++i)
-      if (lane + 32 * i < E) part += exp((double)raw[i] - (double)m);
-    const double den = warp_sum_d(part);
-    gate = (float)(exp((double)sel_raw - (double)m) / den);
+      for (int i = 0; i < NK; ++i) lm = fmaxf(lm, raw[u][i]);
+      const float m = warp_max_f(lm);
+      double part = 0.0;
+#pragma unroll
+      for (int i = 0; i < NK; ++i)
+        if (lane + 32 * i < E) part += exp((double)raw[u][i] - (double)m);
+      const double den = warp_sum_d(part);
+      gate[u] = (float)(exp((double)sel_raw[u] - (double)m) / den);
+    }
   }
+  return nan_tok;
 }
 
 }  // namespace moe

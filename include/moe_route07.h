@@ -58,7 +58,7 @@ typedef enum {
   MOE_ERR_WORKSPACE = 3,      /* workspace NULL, misaligned or too small */
   MOE_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
   MOE_ERR_DEVICE_RANGE = 5,   /* device: expert id or row index out of range */
-  MOE_ERR_DEVICE_TIMEOUT = 6, /* device: a bounded wait in moe_layout gave up */
+  MOE_ERR_DEVICE_TIMEOUT = 6, /* device: a bounded wait gave up */
   MOE_ERR_DEVICE_NAN = 7      /* device: a routing key was NaN */
 } moe_status_t;
 
@@ -98,7 +98,8 @@ int64_t moe_layout_rows(const moe_shape_t* shape);
 size_t moe_workspace_bytes(const moe_shape_t* shape);
 
 /* Zero-fill a workspace (cudaMemsetAsync on `stream`).  Required once before
- * the workspace's first use; every call leaves it ready for the next one. */
+ * the workspace's first use, and again after a call returned MOE_ERR_CUDA;
+ * every successful call leaves it ready for the next one. */
 moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Step 1 -- route ("19. All-to-all", section "Why the router can ruin your
@@ -161,6 +162,18 @@ moe_status_t moe_dispatch(const moe_shape_t* shape, const void* x, const int32_t
                           void* out, float* scales, void* ws, size_t ws_bytes,
                           moe_stream_t stream);
 
+/* Steps 1-4 in one call: moe_route_layout followed by moe_dispatch, with the
+ * same results bit for bit.  Inside this call the dispatch kernel starts
+ * reading rows of x while the layout is still running (x is complete: every
+ * kernel before this call has finished by then), so part of the copy overlaps
+ * the latency-bound layout.  Arguments: the union of the two calls. */
+moe_status_t moe_route_layout_dispatch(const moe_shape_t* shape, const float* logits,
+                                       const float* bias, const void* x, int32_t* ids,
+                                       float* gates, int32_t* counts, int32_t* expert_off,
+                                       int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
+                                       int32_t* src_idx, void* out, float* scales, void* ws,
+                                       size_t ws_bytes, moe_stream_t stream);
+
 /* Step 5 -- combine ("GPU MoE all-to-all", section "Two collectives per
  * layer": the inverse permutation scaled by the router's gate weights; "MoE
  * All-to-All Dispatch and Ragged Routing", section "Returning Tokens to the
@@ -188,19 +201,20 @@ moe_status_t moe_combine(const moe_shape_t* shape, const void* y, const int32_t*
  * Same arguments, results and determinism as moe_layout, minus `ws`.  The
  * scratch lives in a static device array of 256 + MOE_NOALLOC_TABLE_BYTES
  * bytes that every GPU loading the library keeps until the process exits.
- * Limit: ceil(T / 128) * E * 4 <= MOE_NOALLOC_TABLE_BYTES, i.e.
- * ceil(T/128) * E <= 524288 (T = 65536 with E = 1024, T = 131072 with
- * E = 512); larger shapes return MOE_ERR_UNSUPPORTED and launch nothing.
+ * Limit: the layout's two tile tables need 2 * min(ceil(T/16), 128) * E * 4
+ * bytes, so min(ceil(T/16), 128) * E <= 65536 (any T for E <= 512, T <= 1024
+ * for E = 1024); larger shapes return MOE_ERR_UNSUPPORTED and launch nothing.
  * Allocates nothing: no cudaMalloc / cudaFree or allocating library call.
  *  - The first call on a device resolves the array's device address and
  *    zero-fills it (cudaMemsetAsync on `stream`): make that first call before
  *    any stream capture.
- *  - Every call clears the scratch header on `stream` before its kernels.
+ *  - Every call leaves the array ready for the next one; a call whose launch
+ *    fails zero-fills it again.
  *  - All calls share the one array, so calls that overlap on the GPU race;
  *    order them (one stream, or events).
  *  - Device-side problems are not reported (there is no workspace to read
  *    them from); an id outside [0,E) still comes out as dst_pos -1. */
-#define MOE_NOALLOC_TABLE_BYTES (2u << 20)
+#define MOE_NOALLOC_TABLE_BYTES (512u << 10)
 moe_status_t moe_layout_noalloc(const moe_shape_t* shape, const int32_t* ids, int32_t* counts,
                                 int32_t* expert_off, int32_t* rank_off, int32_t* rank_counts,
                                 int32_t* dst_pos, int32_t* src_idx, moe_stream_t stream);

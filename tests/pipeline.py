@@ -68,7 +68,8 @@ def standin_oracle(w: Workload, disp, L):
 
 def run_gpu(w: Workload, inp, ids=None, gates=None, fused=False):
     """Run route (unless ids/gates are given), layout, dispatch, stand-in and
-    combine on cuda:0 (fused: route and layout in one moe_route_layout call).
+    combine on cuda:0.  fused=True: route and layout in one moe_route_layout
+    call; fused="dispatch": steps 1-4 in one moe_route_layout_dispatch call.
     Returns a dict of CUDA tensors and the workspace."""
     import combine_moe_route_07_b200 as m
     dev = torch.device("cuda:0")
@@ -76,7 +77,12 @@ def run_gpu(w: Workload, inp, ids=None, gates=None, fused=False):
     ws = m.Workspace(shape, dev)
     x = inp.x.to(dev)
     res = {"ws": ws, "x": x}
-    if fused:
+    disp = None
+    if fused == "dispatch":
+        logits = inp.logits.to(dev)
+        bias = None if inp.bias is None else inp.bias.to(dev)
+        ids, gates, lay, disp = m.moe_route_layout_dispatch(shape, logits, x, bias, ws=ws)
+    elif fused:
         logits = inp.logits.to(dev)
         bias = None if inp.bias is None else inp.bias.to(dev)
         ids, gates, lay = m.moe_route_layout(shape, logits, bias, ws=ws)
@@ -91,7 +97,8 @@ def run_gpu(w: Workload, inp, ids=None, gates=None, fused=False):
         lay = m.moe_layout(shape, ids, ws=ws)
     res["ids"], res["gates"] = ids, gates
     res["layout"] = lay
-    disp = m.moe_dispatch(shape, x, lay.dst_pos, ws=ws)
+    if disp is None:
+        disp = m.moe_dispatch(shape, x, lay.dst_pos, ws=ws)
     res["dispatch"] = disp
     y = standin_gpu(w, disp, lay)
     res["y"] = y

@@ -65,7 +65,7 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
+@pytest.mark.parametrize("fused", [False, True, "dispatch"], ids=["separate", "fused", "fused3"])
 @pytest.mark.parametrize("w", CASES, ids=[c.name for c in CASES])
 def test_edge_case_parity(w, fused):
     _check_all(w, fused=fused)
@@ -101,7 +101,7 @@ def test_all_tokens_on_the_same_experts():
     bias = torch.zeros(16)
     bias[5], bias[2], bias[7] = 300.0, 200.0, 100.0
     inp.bias = bias
-    for fused in (False, True):
+    for fused in (False, True, "dispatch"):
         _check_all(w, inp, fused)
         wc = w.with_(name="same_experts_capacity", capacity_factor=0.25)
         _check_all(wc, inp, fused)

@@ -31,7 +31,7 @@ def _compare_layout(g_lay, L, what):
         assert np.array_equal(got, L[key]), f"{what}: layout.{key} differs"
 
 
-@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
+@pytest.mark.parametrize("fused", [False, True, "dispatch"], ids=["separate", "fused", "fused3"])
 @pytest.mark.parametrize("name", SMALL)
 def test_full_path_small_configs(name, fused):
     w = WORKLOADS[name]
@@ -73,7 +73,7 @@ def test_each_kernel_on_oracle_inputs(name):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
+@pytest.mark.parametrize("fused", [False, True, "dispatch"], ids=["separate", "fused", "fused3"])
 @pytest.mark.parametrize("name", BIG)
 def test_full_size_route_layout_exact_and_sampled_payload(name, fused):
     import combine_moe_route_07_b200 as m

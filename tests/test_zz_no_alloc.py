@@ -80,8 +80,8 @@ def test_noalloc_matches_workspace_layout_twice(w):
 def test_noalloc_rejects_shapes_beyond_its_limit():
     lib = _binding.lib()
     fake = ctypes.c_void_p(0x1000)
-    # 513 tiles x 1024 experts x 4 bytes > 2 MiB (E = 1024 allows T <= 65536)
-    too_big = Workload("too_big", T=65536 + 128, H=128, E=1024, R=8, k=2)
+    # two tables of 65 tiles x 1024 experts x 4 bytes > 512 KiB (E = 1024 allows T <= 1024)
+    too_big = Workload("too_big", T=1025, H=128, E=1024, R=8, k=2)
     st = lib.moe_layout_noalloc(ctypes.byref(_shape_c(too_big)), fake, fake, fake, fake, fake,
                                 fake, fake, None)
     assert st == _binding.MOE_ERR_UNSUPPORTED
