@@ -162,6 +162,24 @@ def ncu_traffic(kernel, workload):
     return None
 
 
+# ------------------------------------------------------------ multi-rank --
+
+def max_over_ranks(x: float, dist=None, device=None) -> float:
+    """The max of a per-rank scalar (a device time) over all ranks."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(world: int, tokens_per_rank: int, steps: int, max_ms: float) -> float:
+    """Weak scaling: every rank processes its own batch each step; the job's
+    throughput is all ranks' tokens over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (max_ms * 1e-3)
+
+
 # ----------------------------------------------------------------- oracle --
 
 def oracle_step_fn(w, inp, tokens):
@@ -329,7 +347,8 @@ def main():
     m.moe_check(ws)
 
     L2_BYTES = 126 * 10**6
-    touched = sum(algorithmic_bytes(w, kept_rows).values())
+    _b = algorithmic_bytes(w, kept_rows)
+    touched = _b["route"] + _b["layout"] + _b["dispatch"] + _b["combine"]
     flush_between = touched < 2 * L2_BYTES
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush_between else None
 
@@ -419,11 +438,7 @@ def main():
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
     m.moe_check(ws)
-    total_ms = sum(a.elapsed_time(b) for a, b in ev)
-    if dist is not None:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dist, dev)
 
     # per-kernel breakdown: a probe graph of the same step with event-record
     # nodes between the kernels, replayed after an L2 flush and read back one
@@ -468,11 +483,7 @@ def main():
             out_h.copy_(out, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        if dist is not None:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dist, dev)
         e2e = {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": x_h.numel() * 2 + lg_h.numel() * 4,
                "d2h_bytes_per_step": out_h.numel() * 2, "ms_per_step": e2e_ms}
@@ -499,7 +510,7 @@ def main():
     ms_step = total_ms / K
     line = {
         "metric": METRIC,
-        "value": world * T * K / (total_ms * 1e-3),
+        "value": whole_job_tokens_per_s(world, T, K, total_ms),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": K,

@@ -1,0 +1,74 @@
+"""Host-side logic of the multi-GPU bench (replicas, weak scaling), run as two
+gloo ranks on the CPU: the max over ranks and the whole-job throughput."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, times, q):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        m = bench.max_over_ranks(times[rank], dist, "cpu")
+        v = bench.whole_job_tokens_per_s(world, 4096, 10, m)
+        q.put((rank, m, v))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_weak_scaling_value_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    times = [12.5, 17.25]
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, times, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=10) for _ in range(2))
+    for rank, m, v in got:
+        assert m == 17.25  # every rank sees the slowest rank's time
+        assert v == pytest.approx(2 * 4096 * 10 / 17.25e-3)
+
+
+def test_single_rank_is_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.5) == 3.5
+    assert bench.whole_job_tokens_per_s(1, 100, 4, 2.0) == pytest.approx(100 * 4 / 2e-3)
+
+
+def test_reference_arm_prints_one_line_and_other_ranks_stay_silent(capsys, monkeypatch):
+    sys.path.insert(0, ROOT)
+    import json
+    import bench
+    from combine_moe_route_07_b200.workloads import WORKLOADS
+    args = type("A", (), dict(gpus=2, steps=2, warmup=1))()
+    monkeypatch.setenv("RANK", "1")
+    assert bench.run_reference(args, WORKLOADS["tiny"]) == 0
+    assert capsys.readouterr().out == ""
+    monkeypatch.setenv("RANK", "0")
+    assert bench.run_reference(args, WORKLOADS["tiny"]) == 0
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
