@@ -248,7 +248,7 @@ moe_status_t moe_combine(const moe_shape_t* shape, const void* y, const int32_t*
   if (shape->tokens == 0) return MOE_OK;
   return from_cuda(moe::launch_combine(env_of(stream), y, dst_pos, gates, shared, residual,
                                        shape->tokens, shape->hidden, shape->k, rows_of(shape),
-                                       out, static_cast<WsHeader*>(ws)));
+                                       out, static_cast<WsHeader*>(ws), shape->capacity > 0));
 }
 
 moe_status_t moe_get_device_error(void* ws, int32_t* detail, moe_stream_t stream) {

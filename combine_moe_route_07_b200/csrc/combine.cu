@@ -24,8 +24,7 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kBatch = 4;     // slots whose loads are in flight together
-constexpr int kMinBlocks = 4;  // CTAs per SM the register budget must allow
+
 
 __device__ __forceinline__ void fma8(float (&acc)[8], float g, const uint4& v) {
   acc[0] = __fmaf_rn(g, bf16lo(v.x), acc[0]);
@@ -55,9 +54,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // One warp per (token, slice of 32*CPT chunks); lane j < k fetches the row
-// and gate of slot j once and the warp broadcasts them by shuffle.
-template <int CPT>
-__global__ void __launch_bounds__(kThreads, kMinBlocks)
+// and gate of slot j once and the warp broadcasts them by shuffle.  With
+// PF the next task's rows and gates are fetched while this one computes, and
+// a batch of slots that are all dropped issues no loads at all (capacity mode
+// drops most slots of a skewed batch).
+template <int CPT, int KB, int MINB, bool PF>
+__global__ void __launch_bounds__(kThreads, MINB)
     combine_kernel(const char* __restrict__ y, const int32_t* __restrict__ dst_pos,
                    const float* __restrict__ gates, const char* __restrict__ shared,
                    const char* __restrict__ residual, int T, int H, int k, int64_t N,
@@ -70,32 +72,42 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
   const int64_t tasks = (int64_t)T * S;
   const size_t row_bytes = (size_t)H * 2;
   const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
-  for (int64_t task = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5; task < tasks;
-       task += nw) {
-    const int t = (int)(task / S);
-    const int cb = (int)(task - (int64_t)t * S) * 32 * CPT + lane;
-    int pl = -1;
-    float gl = 0.0f;
-    if (lane < k) {
-      pl = __ldg(dst_pos + (size_t)t * k + lane);
-      gl = __ldg(gates + (size_t)t * k + lane);
-      if (pl >= N) {
-        report(hdr, MOE_ERR_DEVICE_RANGE, pl);
-        pl = -1;
+  // slot j of task `task` (lane j < k), -1 when dropped or out of range
+  auto fetch = [&](int64_t task, int& p, float& g) {
+    p = -1;
+    g = 0.0f;
+    if (task < tasks && lane < k) {
+      const int t = (int)((uint32_t)task / (uint32_t)S);  // tasks < 2^31 (host check)
+      p = __ldg(dst_pos + (size_t)t * k + lane);
+      g = __ldg(gates + (size_t)t * k + lane);
+      if (p >= N) {
+        report(hdr, MOE_ERR_DEVICE_RANGE, p);
+        p = -1;
       }
     }
+  };
+  int64_t task = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+  int pl, pn = -1;
+  float gl, gn = 0.0f;
+  fetch(task, pl, gl);
+  for (; task < tasks; task += nw) {
+    if (PF) fetch(task + nw, pn, gn);
+    const int t = (int)((uint32_t)task / (uint32_t)S);
+    const int cb = (int)((uint32_t)task - (uint32_t)t * (uint32_t)S) * 32 * CPT + lane;
+    const unsigned kept = __ballot_sync(kFull, pl >= 0);
     float acc[CPT][8];
 #pragma unroll
     for (int i = 0; i < CPT; ++i)
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[i][e] = 0.0f;
 
-    for (int j0 = 0; j0 < k; j0 += kBatch) {
-      uint4 v[kBatch][CPT];
-      float gw[kBatch];
-      int pp[kBatch];
+    for (int j0 = 0; j0 < k; j0 += KB) {
+      if (((kept >> j0) & ((1u << KB) - 1u)) == 0u) continue;  // every slot dropped
+      uint4 v[KB][CPT];
+      float gw[KB];
+      int pp[KB];
 #pragma unroll
-      for (int jj = 0; jj < kBatch; ++jj) {
+      for (int jj = 0; jj < KB; ++jj) {
         const int j = j0 + jj;  // j < 32: the shuffle source is always a lane
         pp[jj] = __shfl_sync(kFull, pl, j & 31);
         gw[jj] = __shfl_sync(kFull, gl, j & 31);
@@ -111,7 +123,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
         }
       }
 #pragma unroll
-      for (int jj = 0; jj < kBatch; ++jj)
+      for (int jj = 0; jj < KB; ++jj)
         if (pp[jj] >= 0) {
 #pragma unroll
           for (int i = 0; i < CPT; ++i) fma8(acc[i], gw[jj], v[jj][i]);
@@ -132,16 +144,23 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
       o.w = pack_bf16x2(acc[i][6], acc[i][7]);
       st16(out + off, o);
     }
+    if (PF) {
+      pl = pn;
+      gl = gn;
+    } else {
+      fetch(task + nw, pl, gl);
+    }
   }
 }
 
+// Enough CTAs for one warp per task, at most the ones resident at once.
 template <typename K>
-int grid_for(K kernel, const LaunchEnv& env, int64_t units) {
+int grid_for(K kernel, const LaunchEnv& env, int64_t tasks) {
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess ||
       per_sm < 1)
     per_sm = 1;
-  const int64_t need = (units + kThreads - 1) / kThreads;
+  const int64_t need = (tasks + kThreads / 32 - 1) / (kThreads / 32);
   const int64_t cap = (int64_t)env.num_sms * per_sm;
   int64_t g = need < cap ? need : cap;
   return (int)(g < 1 ? 1 : g);
@@ -151,14 +170,26 @@ int grid_for(K kernel, const LaunchEnv& env, int64_t units) {
 
 cudaError_t launch_combine(const LaunchEnv& env, const void* y, const int32_t* dst_pos,
                            const float* gates, const void* shared, const void* residual, int T,
-                           int H, int k, int64_t N, void* out, WsHeader* hdr) {
+                           int H, int k, int64_t N, void* out, WsHeader* hdr, bool sparse) {
   if (T == 0) return cudaSuccess;
   const int C8 = H / 8;
-  auto kern = combine_kernel<1>;
-  const int grid = grid_for(kern, env, (int64_t)T * ((C8 + 31) / 32) * 32);
-  return launch_pdl(env, kern, dim3(grid), dim3(kThreads), 0, static_cast<const char*>(y), dst_pos,
-                    gates, static_cast<const char*>(shared), static_cast<const char*>(residual), T,
-                    H, k, N, static_cast<char*>(out), hdr);
+  const char* ys = static_cast<const char*>(y);
+  const char* sh = static_cast<const char*>(shared);
+  const char* rs = static_cast<const char*>(residual);
+  char* o = static_cast<char*>(out);
+  // Capacity mode drops most slots of a skewed batch: then each task moves
+  // little and its latency dominates, so wider slices with the next task's
+  // metadata prefetched win; dense layouts do better with more warps.
+  if (sparse && C8 >= 128) {
+    auto kern = combine_kernel<4, 2, 2, true>;
+    const int grid = grid_for(kern, env, (int64_t)T * ((C8 + 127) / 128));
+    return launch_pdl(env, kern, dim3(grid), dim3(kThreads), 0, ys, dst_pos, gates, sh, rs, T, H,
+                      k, N, o, hdr);
+  }
+  auto kern = combine_kernel<1, 4, 4, false>;
+  const int grid = grid_for(kern, env, (int64_t)T * ((C8 + 31) / 32));
+  return launch_pdl(env, kern, dim3(grid), dim3(kThreads), 0, ys, dst_pos, gates, sh, rs, T, H, k,
+                    N, o, hdr);
 }
 
 }  // namespace moe

@@ -45,8 +45,8 @@ __global__ void __launch_bounds__(kThreads)
   const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
   for (int64_t task = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5; task < tasks;
        task += nw) {
-    const int t = (int)(task / S);
-    const int cb = (int)(task - (int64_t)t * S) * 32 * CPT + lane;
+    const int t = (int)((uint32_t)task / (uint32_t)S);  // tasks < 2^31 (host check)
+    const int cb = (int)((uint32_t)task - (uint32_t)t * (uint32_t)S) * 32 * CPT + lane;
     const char* src = x + (size_t)t * row_bytes;
     uint4 v[CPT];
 #pragma unroll
@@ -73,11 +73,12 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // Bulk-copy (TMA) variant for rows of 1-32 KiB.  Each CTA runs kBulkWarps
-// independent pipelines; lane 0 of a warp streams its tokens through
-// `stages` shared-memory row buffers: a bulk load global -> shared completes
-// on the stage's mbarrier, then k bulk stores shared -> global (one bulk
-// group per token) write the copies, and the stage is refilled once the
-// previous token's group has finished reading it.  No thread touches the row
+// independent pipelines over units (a token row, or a slice of one when there
+// are too few tokens to keep every SM busy); lane 0 of a warp streams its
+// units through `stages` shared-memory buffers: a bulk load global -> shared
+// completes on the stage's mbarrier, then k bulk stores shared -> global (one
+// bulk group per unit) write the copies, and the stage is refilled once the
+// previous unit's group has finished reading it.  No thread touches the row
 // data, so the LSU carries only the dst_pos loads.  Every wait is bounded.
 constexpr int kBulkWarps = 4;
 constexpr int kBulkMaxStages = 8;
@@ -86,7 +87,8 @@ constexpr uint64_t kBulkTimeoutNs = 1000000000ull;
 __global__ void __launch_bounds__(kBulkWarps * 32)
     dispatch_bf16_bulk_kernel(const char* __restrict__ x, const int32_t* __restrict__ dst_pos,
                               int T, int H, int k, int64_t N, char* __restrict__ out, int stages,
-                              uint32_t stage_bytes, int x_ready, WsHeader* hdr) {
+                              uint32_t stage_bytes, int nsl, uint32_t slice_bytes, int x_ready,
+                              WsHeader* hdr) {
   extern __shared__ __align__(128) unsigned char sbuf[];
   __shared__ uint64_t bars[kBulkWarps][kBulkMaxStages];
   // x_ready: the kernel launched just before this one did not write x, and
@@ -98,7 +100,7 @@ __global__ void __launch_bounds__(kBulkWarps * 32)
     pdl_trigger();
   }
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t row = (uint32_t)H * 2u;
+  const size_t row = (size_t)H * 2;
   unsigned char* st = sbuf + (size_t)w * stages * stage_bytes;
   uint64_t* bar = bars[w];
   if (lane == 0) {
@@ -106,53 +108,64 @@ __global__ void __launch_bounds__(kBulkWarps * 32)
     mbar_fence_init();
   }
   __syncwarp();
+  const int64_t units = (int64_t)T * nsl;
   const int64_t stride = (int64_t)gridDim.x * kBulkWarps;
   const int64_t first = (int64_t)blockIdx.x * kBulkWarps + w;
-  const int64_t count = first < T ? (T - 1 - first) / stride + 1 : 0;
+  const int64_t count = first < units ? (units - 1 - first) / stride + 1 : 0;
+  // unit -> token, byte offset in the row, bytes
+  // units < 2^31 (T * H/8 < 2^31 is checked on the host)
+  auto unit_tok = [&](int64_t i) { return (uint32_t)(first + i * stride) / (uint32_t)nsl; };
+  auto unit_off = [&](int64_t i) {
+    return ((uint32_t)(first + i * stride) % (uint32_t)nsl) * slice_bytes;
+  };
+  auto unit_len = [&](int64_t i) {
+    const uint32_t o = unit_off(i);
+    return (uint32_t)min((size_t)slice_bytes, row - o);
+  };
+  auto issue_load = [&](int64_t i) {
+    const int sn = (int)(i % stages);
+    const uint32_t len = unit_len(i);
+    mbar_arrive_expect_tx(&bar[sn], len);
+    bulk_load(st + (size_t)sn * stage_bytes, x + (size_t)unit_tok(i) * row + unit_off(i), len,
+              &bar[sn]);
+  };
   int64_t issued = 0;  // loads issued (lane 0)
-  if (lane == 0) {
-    for (; issued < count && issued < stages - 1; ++issued) {
-      mbar_arrive_expect_tx(&bar[issued], row);
-      bulk_load(st + (size_t)issued * stage_bytes, x + (size_t)(first + issued * stride) * row,
-                row, &bar[issued]);
-    }
-  }
+  if (lane == 0)
+    for (; issued < count && issued < stages - 1; ++issued) issue_load(issued);
   if (x_ready) {  // dst_pos comes from the kernel launched just before
     pdl_wait();
     pdl_trigger();
   }
   uint32_t parity = 0;  // bit s: the phase stage s completes next
   bool ok = true;
-  int pl = (count > 0 && lane < k) ? __ldg(dst_pos + (size_t)first * k + lane) : -1;
+  int pl = (count > 0 && lane < k) ? __ldg(dst_pos + (size_t)unit_tok(0) * k + lane) : -1;
   for (int64_t i = 0; i < count && ok; ++i) {
     const int s = (int)(i % stages);
     const int p_cur = pl;
-    if (i + 1 < count && lane < k)  // next token's rows, while this one streams
-      pl = __ldg(dst_pos + (size_t)(first + (i + 1) * stride) * k + lane);
+    if (i + 1 < count && lane < k)  // next unit's rows, while this one streams
+      pl = __ldg(dst_pos + (size_t)unit_tok(i + 1) * k + lane);
     if (lane == 0) {
       ok = mbar_wait_bounded(&bar[s], (parity >> s) & 1u, kBulkTimeoutNs);
       parity ^= 1u << s;
-      if (!ok) report(hdr, MOE_ERR_DEVICE_TIMEOUT, (int)(first + i * stride));
+      if (!ok) report(hdr, MOE_ERR_DEVICE_TIMEOUT, (int)unit_tok(i));
     }
     ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
     if (!ok) break;
+    const uint32_t off = unit_off(i), len = unit_len(i);
     for (int j = 0; j < k; ++j) {
       const int p = __shfl_sync(kFull, p_cur, j);
       if (lane == 0 && p >= 0) {
         if (p < N)
-          bulk_store(out + (size_t)p * row, st + (size_t)s * stage_bytes, row);
+          bulk_store(out + (size_t)p * row + off, st + (size_t)s * stage_bytes, len);
         else
           report(hdr, MOE_ERR_DEVICE_RANGE, p);
       }
     }
     if (lane == 0) {
       bulk_commit();
-      if (issued < count) {  // refill the stage token i-1 used
+      if (issued < count) {  // refill the stage unit i-1 used
         bulk_wait_read<1>();
-        const int sn = (int)(issued % stages);
-        mbar_arrive_expect_tx(&bar[sn], row);
-        bulk_load(st + (size_t)sn * stage_bytes, x + (size_t)(first + issued * stride) * row, row,
-                  &bar[sn]);
+        issue_load(issued);
         ++issued;
       }
     }
@@ -161,7 +174,8 @@ __global__ void __launch_bounds__(kBulkWarps * 32)
   if (lane == 0) {
     bulk_wait_all();
     if (!ok) {  // let the loads still in flight land before the CTA exits
-      for (int s = 0; s < stages; ++s) (void)mbar_wait_bounded(&bar[s], (parity >> s) & 1u, kBulkTimeoutNs);
+      for (int s = 0; s < stages; ++s)
+        (void)mbar_wait_bounded(&bar[s], (parity >> s) & 1u, kBulkTimeoutNs);
     }
   }
 }
@@ -193,8 +207,8 @@ __global__ void __launch_bounds__(kThreads)
   const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
   for (int64_t task = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5; task < tasks;
        task += nw) {
-    const int t = (int)(task / S);
-    const int cb = (int)(task - (int64_t)t * S) * 32 * CPT + lane;
+    const int t = (int)((uint32_t)task / (uint32_t)S);  // tasks < 2^31 (host check)
+    const int cb = (int)((uint32_t)task - (uint32_t)t * (uint32_t)S) * 32 * CPT + lane;
     const char* src = x + (size_t)t * row_bytes;
     uint32_t q[CPT][2];
     float s[CPT];
@@ -268,7 +282,16 @@ cudaError_t launch_dispatch_bf16(const LaunchEnv& env, const void* x, const int3
   char* o = static_cast<char*>(out);
   const uint32_t row = (uint32_t)H * 2u;
   if (row >= 1024 && row <= 32768) {
-    const uint32_t stage_bytes = (row + 127u) & ~127u;
+    const int64_t warps = (int64_t)env.num_sms * kBulkWarps;  // one CTA per SM
+    // slices of >= 1 KiB (16-byte multiples) when the tokens alone cannot
+    // give every pipeline two units
+    int64_t nsl = (2 * warps + T - 1) / T;
+    const int64_t max_nsl = row / 1024;
+    if (nsl > max_nsl) nsl = max_nsl;
+    if (nsl < 1) nsl = 1;
+    const uint32_t slice = (uint32_t)((((row + nsl - 1) / nsl) + 15) / 16 * 16);
+    nsl = (row + slice - 1) / slice;
+    const uint32_t stage_bytes = (slice + 127u) & ~127u;
     int stages = (int)((200u * 1024u) / (kBulkWarps * stage_bytes));
     if (stages > kBulkMaxStages) stages = kBulkMaxStages;
     if (stages >= 2) {
@@ -282,11 +305,11 @@ cudaError_t launch_dispatch_bf16(const LaunchEnv& env, const void* x, const int3
       if (err != cudaSuccess) return err;
       if (per_sm < 1) per_sm = 1;
       int64_t grid = (int64_t)per_sm * env.num_sms;
-      const int64_t need = ((int64_t)T + kBulkWarps - 1) / kBulkWarps;
+      const int64_t need = ((int64_t)T * nsl + kBulkWarps - 1) / kBulkWarps;
       if (grid > need) grid = need;
       return launch_pdl(env, dispatch_bf16_bulk_kernel, dim3((unsigned)grid),
                         dim3(kBulkWarps * 32), smem, xs, dst_pos, T, H, k, N, o, stages,
-                        stage_bytes, x_ready ? 1 : 0, hdr);
+                        stage_bytes, (int)nsl, slice, x_ready ? 1 : 0, hdr);
     }
   }
   if (C8 >= 256) {

@@ -87,8 +87,9 @@ cudaError_t launch_dispatch_fp8(const LaunchEnv& env, const void* x, const int32
                                 int T, int H, int k, int64_t N, void* out, float* scales,
                                 WsHeader* hdr);
 
+// sparse: most slots may be dropped (capacity mode)
 cudaError_t launch_combine(const LaunchEnv& env, const void* y, const int32_t* dst_pos,
                            const float* gates, const void* shared, const void* residual, int T,
-                           int H, int k, int64_t N, void* out, WsHeader* hdr);
+                           int H, int k, int64_t N, void* out, WsHeader* hdr, bool sparse);
 
 }  // namespace moe
