@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(kBulkWarps * 32)
     dispatch_bf16_bulk_kernel(const char* __restrict__ x, const int32_t* __restrict__ dst_pos,
                               int T, int H, int k, int64_t N, char* __restrict__ out, int stages,
                               uint32_t stage_bytes, int nsl, uint32_t slice_bytes, int x_ready,
-                              WsHeader* hdr) {
+                              int evict_first, WsHeader* hdr) {
   extern __shared__ __align__(128) unsigned char sbuf[];
   __shared__ uint64_t bars[kBulkWarps][kBulkMaxStages];
   // x_ready: the kernel launched just before this one did not write x, and
@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(kBulkWarps * 32)
   }
   uint32_t parity = 0;  // bit s: the phase stage s completes next
   bool ok = true;
+  const uint64_t pol = l2_evict_first_policy();
   int pl = (count > 0 && lane < k) ? __ldg(dst_pos + (size_t)unit_tok(0) * k + lane) : -1;
   for (int64_t i = 0; i < count && ok; ++i) {
     const int s = (int)(i % stages);
@@ -156,7 +157,10 @@ __global__ void __launch_bounds__(kBulkWarps * 32)
       const int p = __shfl_sync(kFull, p_cur, j);
       if (lane == 0 && p >= 0) {
         if (p < N)
-          bulk_store(out + (size_t)p * row + off, st + (size_t)s * stage_bytes, len);
+          if (evict_first)  // output larger than L2: let its lines go back to DRAM early
+            bulk_store_hint(out + (size_t)p * row + off, st + (size_t)s * stage_bytes, len, pol);
+          else
+            bulk_store(out + (size_t)p * row + off, st + (size_t)s * stage_bytes, len);
         else
           report(hdr, MOE_ERR_DEVICE_RANGE, p);
       }
@@ -307,9 +311,13 @@ cudaError_t launch_dispatch_bf16(const LaunchEnv& env, const void* x, const int3
       int64_t grid = (int64_t)per_sm * env.num_sms;
       const int64_t need = ((int64_t)T * nsl + kBulkWarps - 1) / kBulkWarps;
       if (grid > need) grid = need;
+      // an output several times the 126 MB L2 cannot stay there for the next
+      // kernel anyway: mark its lines evict-first so they are written back
+      // while this kernel runs rather than during the next one
+      const int evict_first = ((int64_t)T * k * row > (int64_t)192 << 20) ? 1 : 0;
       return launch_pdl(env, dispatch_bf16_bulk_kernel, dim3((unsigned)grid),
                         dim3(kBulkWarps * 32), smem, xs, dst_pos, T, H, k, N, o, stages,
-                        stage_bytes, (int)nsl, slice, x_ready ? 1 : 0, hdr);
+                        stage_bytes, (int)nsl, slice, x_ready ? 1 : 0, evict_first, hdr);
     }
   }
   if (C8 >= 256) {

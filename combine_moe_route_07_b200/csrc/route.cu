@@ -20,6 +20,7 @@ __global__ void __launch_bounds__(kThreads)
                  int k, int renorm, int32_t* __restrict__ ids, float* __restrict__ gates,
                  WsHeader* hdr, uint32_t* __restrict__ tables, int TT, size_t table_words) {
   extern __shared__ int32_t hist[];  // [E] (HIST)
+  __shared__ uint32_t cand_all[kWarps][NK >= 8 ? 3 * kMaxCand : 1];
   pdl_wait();  // logits (and the tile table) may come from the kernel launched before
   pdl_trigger();
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -37,7 +38,11 @@ __global__ void __launch_bounds__(kThreads)
     if (t < T) {
       int tok[1] = {t}, e[1];
       float g[1];
-      const int nan_tok = route_tokens<NK, 1>(logits, tok, T, b, E, k, renorm, lane, e, g);
+      int nan_tok;
+      if constexpr (NK >= 8)
+        nan_tok = route_token_thr<NK>(logits, t, T, b, E, k, renorm, lane, cand_all[w], e[0], g[0]);
+      else
+        nan_tok = route_tokens<NK, 1>(logits, tok, T, b, E, k, renorm, lane, e, g);
       if (nan_tok >= 0 && lane == 0) report(hdr, MOE_ERR_DEVICE_NAN, nan_tok);
       if (lane < k) {
         ids[(size_t)t * k + lane] = e[0];

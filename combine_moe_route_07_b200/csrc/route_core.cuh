@@ -1,6 +1,5 @@
-// route_core.cuh -- top-k selection and gates for a few tokens at once, one
-// warp per group.  Shared by the standalone route kernel and the fused
-// route + layout kernel.
+// route_core.cuh -- top-k selection and gates, one warp per token (or per
+// group of tokens): the device side of step 1, used by route.cu.
 //
 // "19. All-to-all" (ai-from-scratch), section "Why the router can ruin your
 // day": the per-expert balancing bias enters the top-k decision and nothing
@@ -141,6 +140,140 @@ __device__ __forceinline__ int route_tokens(const float* __restrict__ logits, co
       const double den = warp_sum_d(part);
       gate[u] = (float)(exp((double)sel_raw[u] - (double)m) / den);
     }
+  }
+  return nan_tok;
+}
+
+
+// Exact top-k through a threshold, for many keys per lane (NK >= 8).
+// tau = the k-th largest of the 32 lane maxima: those k maxima are k distinct
+// keys >= tau, so the k-th largest key is >= tau and no key below tau can be
+// selected.  The warp compacts the keys >= tau (usually k to 2k of them) into
+// shared memory and runs the k selection rounds over at most two per lane.
+// More than kMaxCand candidates (heavy ties) falls back to route_tokens.
+// `cand` is this warp's 3*kMaxCand words of shared memory.
+constexpr int kMaxCand = 64;
+
+template <int NK>
+__device__ __forceinline__ int route_token_thr(const float* __restrict__ logits, int t, int T,
+                                               const float (&b)[NK], int E, int k, int renorm,
+                                               int lane, uint32_t* cand, int& sel_e,
+                                               float& gate) {
+  float raw[NK];
+  uint32_t code[NK];
+  bool bad = false;
+  const float* row = logits + (size_t)t * E;
+#pragma unroll
+  for (int i = 0; i < NK; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E) {
+      raw[i] = __ldcs(row + e);
+      const float key = __fadd_rn(raw[i], b[i]);
+      bad |= (key != key);
+      code[i] = order_code(key);
+    } else {
+      raw[i] = -INFINITY;
+      code[i] = 0u;
+    }
+  }
+  const int nan_tok = __any_sync(kFull, bad) ? t : -1;
+
+  // threshold: k-th largest lane maximum
+  uint32_t mm = 0u;
+#pragma unroll
+  for (int i = 0; i < NK; ++i) mm = max(mm, code[i]);
+  uint32_t tau = 0u;
+  for (int j = 0; j < k; ++j) {
+    const uint32_t top = __reduce_max_sync(kFull, mm);
+    tau = top;
+    const unsigned hold = __ballot_sync(kFull, mm == top);
+    if (lane == __ffs(hold) - 1) mm = 0u;
+  }
+  int c = 0;
+#pragma unroll
+  for (int i = 0; i < NK; ++i) c += (code[i] != 0u && code[i] >= tau) ? 1 : 0;
+  const int total = (int)__reduce_add_sync(kFull, (unsigned)c);
+  if (total > kMaxCand) {  // heavy ties at the threshold: the full scan
+    int tok[1] = {t}, e1[1];
+    float g1[1];
+    route_tokens<NK, 1>(logits, tok, T, b, E, k, renorm, lane, e1, g1);
+    sel_e = e1[0];
+    gate = g1[0];
+    return nan_tok;
+  }
+  int pre = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, pre, o);
+    if (lane >= o) pre += y;
+  }
+  pre -= c;
+#pragma unroll
+  for (int i = 0; i < NK; ++i)
+    if (code[i] != 0u && code[i] >= tau) {
+      cand[pre] = code[i];
+      cand[kMaxCand + pre] = (uint32_t)(lane + 32 * i);
+      cand[2 * kMaxCand + pre] = __float_as_uint(raw[i]);
+      ++pre;
+    }
+  __syncwarp();
+  uint32_t c0 = 0u, c1 = 0u, e0 = 0u, e1 = 0u;
+  float r0 = 0.0f, r1 = 0.0f;
+  if (lane < total) {
+    c0 = cand[lane];
+    e0 = cand[kMaxCand + lane];
+    r0 = __uint_as_float(cand[2 * kMaxCand + lane]);
+  }
+  if (lane + 32 < total) {
+    c1 = cand[lane + 32];
+    e1 = cand[kMaxCand + lane + 32];
+    r1 = __uint_as_float(cand[2 * kMaxCand + lane + 32]);
+  }
+  __syncwarp();  // the next token may overwrite cand
+
+  float sel_raw = 0.0f;
+  sel_e = 0;
+  for (int j = 0; j < k; ++j) {
+    const bool use1 = (c1 > c0) || (c1 == c0 && c1 != 0u && e1 < e0);
+    const uint32_t bk = use1 ? c1 : c0;
+    const uint32_t be = use1 ? e1 : e0;
+    const uint32_t top = __reduce_max_sync(kFull, bk);
+    const uint32_t win = __reduce_min_sync(kFull, (bk == top) ? be : 0xffffffffu);
+    const bool mine = (bk == top) && (be == win);
+    float r = 0.0f;
+    if (mine) {
+      if (use1) {
+        c1 = 0u;
+        r = r1;
+      } else {
+        c0 = 0u;
+        r = r0;
+      }
+    }
+    const unsigned holder = __ballot_sync(kFull, mine);
+    r = __shfl_sync(kFull, r, __ffs(holder) - 1);
+    if (lane == j) {
+      sel_e = (int)win;
+      sel_raw = r;
+    }
+  }
+
+  if (renorm) {
+    const float m = warp_max_f(lane < k ? sel_raw : -INFINITY);
+    const double ex = (lane < k) ? exp((double)sel_raw - (double)m) : 0.0;
+    const double den = warp_sum_d(ex);
+    gate = (float)(ex / den);
+  } else {
+    float lm = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < NK; ++i) lm = fmaxf(lm, raw[i]);
+    const float m = warp_max_f(lm);
+    double part = 0.0;
+#pragma unroll
+    for (int i = 0; i < NK; ++i)
+      if (lane + 32 * i < E) part += exp((double)raw[i] - (double)m);
+    const double den = warp_sum_d(part);
+    gate = (float)(exp((double)sel_raw - (double)m) / den);
   }
   return nan_tok;
 }

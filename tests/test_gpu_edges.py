@@ -107,6 +107,17 @@ def test_all_tokens_on_the_same_experts():
         _check_all(wc, inp, fused)
 
 
+@pytest.mark.parametrize("E,k", [(256, 8), (512, 10), (1024, 32)])
+def test_heavy_ties_take_the_full_scan(E, k):
+    """Keys with few distinct values: the threshold selection sees more than
+    64 candidates and must fall back to the full scan; ties go to the lower id."""
+    w = Workload(f"ties_{E}", T=300, H=16, E=E, R=8, k=k)
+    inp = make_inputs(w)
+    inp.logits = torch.round(inp.logits * 2) / 2
+    inp.logits[:50] = 0.0  # all keys equal
+    _check_all(w, inp)
+
+
 def test_bad_ids_set_the_device_error_and_are_dropped():
     import combine_moe_route_07_b200 as m
     from combine_moe_route_07_b200._binding import MOE_ERR_DEVICE_RANGE
