@@ -263,6 +263,85 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// FP8 with bulk stores, for H a multiple of 512 and rows of at most 8 KiB of
+// codes: each warp streams its tokens; lane l quantises channels
+// 512g + 16l .. +16 of every 512-channel group g (a 128-channel block is 8
+// aligned lanes, its amax a 3-step xor shuffle), writes the codes and scales
+// into one of kFp8Stages shared-memory stages, and lane 0 issues the k bulk
+// stores of the codes row and of the scales row (one bulk group per token).
+constexpr int kFp8Stages = 4;
+
+__global__ void __launch_bounds__(kBulkWarps * 32)
+    dispatch_fp8_bulk_kernel(const char* __restrict__ x, const int32_t* __restrict__ dst_pos,
+                             int T, int H, int k, int64_t N, uint8_t* __restrict__ out,
+                             float* __restrict__ scales, uint32_t stage_bytes, WsHeader* hdr) {
+  extern __shared__ __align__(128) unsigned char sbuf[];
+  pdl_wait();  // x and dst_pos may come from the kernel launched just before
+  pdl_trigger();
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  unsigned char* st = sbuf + (size_t)w * kFp8Stages * stage_bytes;
+  const int groups = H >> 9;  // 512-channel groups
+  const uint32_t srow = (uint32_t)H >> 5;  // bytes of one scales row (H/128 floats)
+  const size_t xrow = (size_t)H * 2;
+  const int64_t stride = (int64_t)gridDim.x * kBulkWarps;
+  int64_t t = (int64_t)blockIdx.x * kBulkWarps + w;
+  int pl = (t < T && lane < k) ? __ldg(dst_pos + (size_t)t * k + lane) : -1;
+  for (int64_t i = 0; t < T; ++i, t += stride) {
+    const int s = (int)(i % kFp8Stages);
+    unsigned char* sp = st + (size_t)s * stage_bytes;
+    const int p_cur = pl;
+    if (t + stride < T && lane < k) pl = __ldg(dst_pos + (size_t)(t + stride) * k + lane);
+    // the stores issued from this stage kFp8Stages tokens ago have read it
+    if (lane == 0) bulk_wait_read<kFp8Stages - 1>();
+    __syncwarp();
+    const char* src = x + (size_t)t * xrow;
+#pragma unroll 4
+    for (int g = 0; g < groups; ++g) {
+      const int ch = 512 * g + 16 * lane;
+      const uint4 v0 = ld16_stream(src + (size_t)ch * 2);
+      const uint4 v1 = ld16_stream(src + (size_t)ch * 2 + 16);
+      float f[16] = {bf16lo(v0.x), bf16hi(v0.x), bf16lo(v0.y), bf16hi(v0.y),
+                     bf16lo(v0.z), bf16hi(v0.z), bf16lo(v0.w), bf16hi(v0.w),
+                     bf16lo(v1.x), bf16hi(v1.x), bf16lo(v1.y), bf16hi(v1.y),
+                     bf16lo(v1.z), bf16hi(v1.z), bf16lo(v1.w), bf16hi(v1.w)};
+      float amax = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(f[e]));
+#pragma unroll
+      for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+      uint4 q = make_uint4(0, 0, 0, 0);
+      float scale = 0.0f;
+      if (amax > 0.0f) {
+        const float inv = __fdiv_rn(448.0f, amax);
+        scale = __fdiv_rn(amax, 448.0f);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) f[e] = __fmul_rn(f[e], inv);
+        q.x = pack_e4m3x4(f[0], f[1], f[2], f[3]);
+        q.y = pack_e4m3x4(f[4], f[5], f[6], f[7]);
+        q.z = pack_e4m3x4(f[8], f[9], f[10], f[11]);
+        q.w = pack_e4m3x4(f[12], f[13], f[14], f[15]);
+      }
+      *reinterpret_cast<uint4*>(sp + ch) = q;
+      if ((lane & 7) == 0) *reinterpret_cast<float*>(sp + H + 4 * (ch >> 7)) = scale;
+    }
+    fence_proxy_async_smem();  // these shared-memory writes before the bulk stores
+    __syncwarp();
+    for (int j = 0; j < k; ++j) {
+      const int p = __shfl_sync(kFull, p_cur, j);
+      if (lane == 0 && p >= 0) {
+        if (p < N) {
+          bulk_store(out + (size_t)p * H, sp, (uint32_t)H);
+          bulk_store(reinterpret_cast<unsigned char*>(scales) + (size_t)p * srow, sp + H, srow);
+        } else {
+          report(hdr, MOE_ERR_DEVICE_RANGE, p);
+        }
+      }
+    }
+    if (lane == 0) bulk_commit();
+  }
+  if (lane == 0) bulk_wait_all();
+}
+
 template <typename K>
 int grid_for(K kernel, const LaunchEnv& env, int64_t units) {
   int per_sm = 0;
@@ -336,6 +415,27 @@ cudaError_t launch_dispatch_fp8(const LaunchEnv& env, const void* x, const int32
                                 WsHeader* hdr) {
   if (T == 0) return cudaSuccess;
   const int C8 = H / 8;
+  // bulk stores need 16-byte multiples: the scales row (H/32 bytes) asks for
+  // H % 512 == 0, and a 16-byte aligned scales buffer
+  if ((H % 512) == 0 && H <= 8192 && (reinterpret_cast<uintptr_t>(scales) & 15u) == 0 &&
+      (reinterpret_cast<uintptr_t>(out) & 15u) == 0) {
+    const uint32_t stage_bytes = (uint32_t)(((size_t)H + H / 32 + 127) / 128 * 128);
+    const size_t smem = (size_t)kBulkWarps * kFp8Stages * stage_bytes;
+    cudaError_t err = cudaFuncSetAttribute(dispatch_fp8_bulk_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dispatch_fp8_bulk_kernel,
+                                                        kBulkWarps * 32, smem);
+    if (err != cudaSuccess) return err;
+    if (per_sm < 1) per_sm = 1;
+    int64_t grid = (int64_t)per_sm * env.num_sms;
+    const int64_t need = ((int64_t)T + kBulkWarps - 1) / kBulkWarps;
+    if (grid > need) grid = need;
+    return launch_pdl(env, dispatch_fp8_bulk_kernel, dim3((unsigned)grid), dim3(kBulkWarps * 32),
+                      smem, static_cast<const char*>(x), dst_pos, T, H, k, N,
+                      static_cast<uint8_t*>(out), scales, stage_bytes, hdr);
+  }
   auto kern = dispatch_fp8_kernel<1>;
   const int grid = grid_for(kern, env, (int64_t)T * ((C8 + 31) / 32) * 32);
   return launch_pdl(env, kern, dim3(grid), dim3(kThreads), 0, static_cast<const char*>(x), dst_pos,

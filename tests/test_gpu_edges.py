@@ -50,6 +50,12 @@ CASES = [
     Workload("fp8_h128", T=333, H=128, E=16, R=4, k=4, fp8=True, expert="dequant"),
     Workload("fp8_capacity", T=400, H=256, E=8, R=2, k=2, fp8=True, expert="dequant",
              capacity_factor=1, residual=True),
+    # H % 512 == 0: the FP8 path that stages codes and scales in shared memory
+    Workload("fp8_bulk_h512", T=137, H=512, E=16, R=4, k=3, fp8=True, expert="dequant"),
+    Workload("fp8_bulk_h1536_capacity", T=300, H=1536, E=8, R=2, k=4, fp8=True,
+             expert="dequant", capacity_factor=0.5, residual=True),
+    Workload("fp8_bulk_h8192", T=41, H=8192, E=8, R=2, k=2, fp8=True, expert="dequant"),
+    Workload("fp8_h8704", T=19, H=8704, E=8, R=2, k=2, fp8=True, expert="dequant"),
     Workload("align128", T=700, H=32, E=16, R=4, k=2, align=128),
     Workload("align3_odd", T=77, H=16, E=6, R=3, k=2, align=3),
     Workload("capacity_c1", T=300, H=16, E=64, R=8, k=4, capacity_factor=0.0001),
@@ -105,6 +111,19 @@ def test_all_tokens_on_the_same_experts():
         _check_all(w, inp, fused)
         wc = w.with_(name="same_experts_capacity", capacity_factor=0.25)
         _check_all(wc, inp, fused)
+
+
+@pytest.mark.parametrize("H", [256, 1024])
+def test_fp8_zero_blocks_get_zero_codes_and_scale(H):
+    """A 128-channel block that is all zeros (or all -0) quantises to code 0
+    and scale 0; its neighbours in the same row are unaffected."""
+    w = Workload(f"fp8_zero_{H}", T=200, H=H, E=16, R=4, k=3, fp8=True, expert="dequant")
+    inp = make_inputs(w)
+    inp.x[::3, :128] = 0.0
+    inp.x[1::7, 128:256] = -0.0
+    inp.x[5] = 0.0
+    for fused in (False, "dispatch"):
+        _check_all(w, inp, fused)
 
 
 @pytest.mark.parametrize("E,k", [(256, 8), (512, 10), (1024, 32)])
