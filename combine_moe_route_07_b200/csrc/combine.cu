@@ -9,13 +9,19 @@
 // section "Why the router can ruin your day": a dropped slot counts as if the
 // token skipped that expert.
 //
-// Token-major gather, HBM-bound.  Each warp owns a 32*CPT-chunk slice of one
-// token row; each lane issues the 16-byte loads of up to kBatch slots before
-// using any of them (independent loads in flight), then accumulates in fp32
-// in slot order j = 0..k-1 with explicit round-to-nearest FMAs, adds the
-// shared-expert row and the residual row, and rounds to bf16 once.
+// Token-major gather, HBM-bound.  Every variant accumulates in fp32 in slot
+// order j = 0..k-1 with round-to-nearest fused multiply-adds, adds the
+// shared-expert row and then the residual row, and rounds to bf16 once, so all
+// of them give the same bits.
+//
+// Register variant: each warp owns a 32*CPT-chunk slice of one token row; each
+// lane issues the 16-byte loads of up to KB slots before using any of them.
+// Bulk variant (dense layouts with many row slices per warp): the row slices
+// arrive in shared memory by bulk copy (TMA), several tokens ahead of the
+// arithmetic, so the bytes in flight do not cost registers.
 #include <cuda_bf16.h>
 
+#include "bulk.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -51,6 +57,22 @@ __device__ __forceinline__ void add8(float (&acc)[8], const uint4& v) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half)
   return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Two fp32 fused multiply-adds in one instruction (sm_100): acc[i] = g * x[i]
+// + acc[i], each rounded to nearest like __fmaf_rn.
+__device__ __forceinline__ void fma8_x2(float (&acc)[8], float g, const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint64_t gg;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(gg) : "f"(g));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint64_t a, x, d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(acc[2 * i]), "f"(acc[2 * i + 1]));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "r"(w[i] << 16), "r"(w[i] & 0xffff0000u));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(gg), "l"(x), "l"(a));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(acc[2 * i]), "=f"(acc[2 * i + 1]) : "l"(d));
+  }
 }
 
 // One warp per (token, slice of 32*CPT chunks); lane j < k fetches the row
@@ -153,12 +175,165 @@ __global__ void __launch_bounds__(kThreads, MINB)
   }
 }
 
+// Bulk variant.  One CTA of kBulkWarps warps per SM; warp w owns a contiguous
+// range of units (token t, 512-byte slice s of the row), so consecutive units
+// mostly share a token and its dst_pos/gates (fetched one token ahead).  Per
+// warp, a ring of `ns` shared-memory stages each holds one unit: the kept
+// slots' slices of y, then the shared-expert and residual slices.  Unit u+ns-1
+// is issued (lanes j < k each start one bulk copy of slot j; lanes 0 and 1 the
+// shared and residual slices) before the warp waits for unit u, so ns-1 units
+// are in flight while it computes.  Lane l computes the 16-byte chunk l of the
+// slice.  Waits are bounded: a stage that does not fill within a second sets
+// MOE_ERR_DEVICE_TIMEOUT, and the warp waits (bounded) for its copies still in
+// flight before it exits.
+constexpr int kBulkWarps = 16;
+constexpr int kBulkMaxStages = 8;
+constexpr uint32_t kBulkSlice = 512;
+constexpr size_t kBulkSmemBudget = 200u * 1024u;
+constexpr uint64_t kBulkTimeoutNs = 1000000000ull;
+
+template <int KMAX>
+__global__ void __launch_bounds__(kBulkWarps * 32, 1)
+    combine_bulk_kernel(const char* __restrict__ y, const int32_t* __restrict__ dst_pos,
+                        const float* __restrict__ gates, const char* __restrict__ shared,
+                        const char* __restrict__ residual, int T, int H, int k, int64_t N,
+                        char* __restrict__ out, WsHeader* hdr, int ns, uint32_t stage_bytes) {
+  extern __shared__ __align__(128) unsigned char sbuf[];
+  __shared__ uint64_t bars[kBulkWarps][kBulkMaxStages];
+  __shared__ float sgate[kBulkWarps][kBulkMaxStages][32];  // gate of each slot, per stage
+  __shared__ uint32_t skept[kBulkWarps][kBulkMaxStages];   // kept-slot mask, per stage
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t row = (uint32_t)H * 2;
+  const int nsl = (int)((row + kBulkSlice - 1) / kBulkSlice);
+  const int extra = (shared != nullptr) + (residual != nullptr);
+  unsigned char* ring = sbuf + (size_t)w * ns * stage_bytes;
+  uint64_t* bar = bars[w];
+  if (lane == 0) {
+    for (int s = 0; s < ns; ++s) mbar_init(&bar[s], 1);
+    mbar_fence_init();
+  }
+  __syncwarp();
+  pdl_wait();  // y, gates and dst_pos may come from the kernel launched just before
+  pdl_trigger();
+  const int64_t units = (int64_t)T * nsl;
+  const int64_t nwarps = (int64_t)gridDim.x * kBulkWarps;
+  const int64_t wid = (int64_t)blockIdx.x * kBulkWarps + w;
+  const int64_t u0 = units * wid / nwarps, u1 = units * (wid + 1) / nwarps;
+  if (u0 >= u1) return;
+  const int nunits = (int)(u1 - u0);
+  const int t0 = (int)(u0 / nsl), sl0 = (int)(u0 - (int64_t)t0 * nsl);
+
+  // issue side: token it, slice isl, stage is; slots of token it (ip, ig)
+  // and of token it+1 (np, ng, checked when they are used)
+  int it = t0, isl = sl0, is = 0;
+  int ip = -1, np = -1;
+  float ig = 0.0f, ng = 0.0f;
+  if (lane < k) {
+    ip = __ldg(dst_pos + (size_t)t0 * k + lane);
+    ig = __ldg(gates + (size_t)t0 * k + lane);
+    if (t0 + 1 < T) {
+      np = __ldg(dst_pos + (size_t)(t0 + 1) * k + lane);
+      ng = __ldg(gates + (size_t)(t0 + 1) * k + lane);
+    }
+  }
+  if (ip >= N) {
+    report(hdr, MOE_ERR_DEVICE_RANGE, ip);
+    ip = -1;
+  }
+  auto issue = [&]() {
+    const uint32_t off = (uint32_t)isl * kBulkSlice;
+    const uint32_t len = min(kBulkSlice, row - off);
+    const unsigned kept = __ballot_sync(kFull, ip >= 0);
+    sgate[w][is][lane] = ig;
+    if (lane == 0) {
+      skept[w][is] = kept;
+      mbar_arrive_expect_tx(&bar[is], ((uint32_t)__popc(kept) + (uint32_t)extra) * len);
+    }
+    __syncwarp();
+    unsigned char* sp = ring + (size_t)is * stage_bytes;
+    if (ip >= 0) bulk_load(sp + (size_t)lane * kBulkSlice, y + (size_t)ip * row + off, len, &bar[is]);
+    if (lane == 0 && shared != nullptr)
+      bulk_load(sp + (size_t)k * kBulkSlice, shared + (size_t)it * row + off, len, &bar[is]);
+    if (lane == 1 && residual != nullptr)
+      bulk_load(sp + (size_t)(k + extra - 1) * kBulkSlice, residual + (size_t)it * row + off, len,
+                &bar[is]);
+    if (++is == ns) is = 0;
+    if (++isl == nsl) {
+      isl = 0;
+      ++it;
+      ip = np;
+      ig = ng;
+      if (ip >= N) {
+        report(hdr, MOE_ERR_DEVICE_RANGE, ip);
+        ip = -1;
+      }
+      np = -1;
+      ng = 0.0f;
+      if (it + 1 < T && lane < k) {
+        np = __ldg(dst_pos + (size_t)(it + 1) * k + lane);
+        ng = __ldg(gates + (size_t)(it + 1) * k + lane);
+      }
+    }
+  };
+
+  int issued = 0;
+  for (; issued < nunits && issued < ns - 1; ++issued) issue();
+  int ct = t0, csl = sl0, cs = 0;
+  uint32_t parity = 0;  // bit s: phase parity stage s waits for next
+  for (int u = 0; u < nunits; ++u) {
+    // the stage of unit u-1 is free again: refill it with unit u+ns-1
+    if (issued < nunits) {
+      issue();
+      ++issued;
+    }
+    const bool ok = mbar_wait_bounded(&bar[cs], (parity >> cs) & 1u, kBulkTimeoutNs);
+    if (!__all_sync(kFull, ok)) {
+      if (lane == 0) report(hdr, MOE_ERR_DEVICE_TIMEOUT, ct);
+      int s2 = cs;  // let the copies still in flight land before the warp exits
+      for (int v = u; v < issued; ++v) {
+        (void)mbar_wait_bounded(&bar[s2], (parity >> s2) & 1u, kBulkTimeoutNs);
+        parity ^= 1u << s2;
+        if (++s2 == ns) s2 = 0;
+      }
+      return;
+    }
+    parity ^= 1u << cs;
+    const uint32_t off = (uint32_t)csl * kBulkSlice;
+    const uint32_t len = min(kBulkSlice, row - off);
+    if ((uint32_t)lane * 16 < len) {
+      const unsigned kept = skept[w][cs];
+      const unsigned char* sp = ring + (size_t)cs * stage_bytes + lane * 16;
+      float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (j < k && ((kept >> j) & 1u))
+          fma8_x2(acc, sgate[w][cs][j],
+                  *reinterpret_cast<const uint4*>(sp + (size_t)j * kBulkSlice));
+      if (shared != nullptr)
+        add8(acc, *reinterpret_cast<const uint4*>(sp + (size_t)k * kBulkSlice));
+      if (residual != nullptr)
+        add8(acc, *reinterpret_cast<const uint4*>(sp + (size_t)(k + extra - 1) * kBulkSlice));
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      st16(out + (size_t)ct * row + off + lane * 16, o);
+    }
+    __syncwarp();  // every lane is done with stage cs before it is refilled
+    if (++cs == ns) cs = 0;
+    if (++csl == nsl) {
+      csl = 0;
+      ++ct;
+    }
+  }
+}
+
 // Enough CTAs for one warp per task, at most the ones resident at once.
 template <typename K>
 int grid_for(K kernel, const LaunchEnv& env, int64_t tasks) {
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess ||
-      per_sm < 1)
+  int per_sm = 1;
+  if (blocks_per_sm(reinterpret_cast<const void*>(kernel), kThreads, 0, &per_sm) != cudaSuccess)
     per_sm = 1;
   const int64_t need = (tasks + kThreads / 32 - 1) / (kThreads / 32);
   const int64_t cap = (int64_t)env.num_sms * per_sm;
@@ -177,6 +352,25 @@ cudaError_t launch_combine(const LaunchEnv& env, const void* y, const int32_t* d
   const char* sh = static_cast<const char*>(shared);
   const char* rs = static_cast<const char*>(residual);
   char* o = static_cast<char*>(out);
+  // Dense layouts with at least 8 row slices per warp of a full bulk grid:
+  // the bulk variant, when the stages of up to 12 slots (k plus the shared
+  // and residual rows) fit twice per warp.
+  const int extra = (shared != nullptr) + (residual != nullptr);
+  const uint32_t stage_bytes = (uint32_t)(k + extra) * kBulkSlice;
+  const int ns_fit = (int)(kBulkSmemBudget / ((size_t)kBulkWarps * stage_bytes));
+  const int64_t slices = (int64_t)T * ((2 * (int64_t)H + kBulkSlice - 1) / kBulkSlice);
+  if (!sparse && k <= 16 && ns_fit >= 2 &&
+      slices >= 8 * (int64_t)env.num_sms * kBulkWarps) {
+    const int ns = ns_fit < kBulkMaxStages ? ns_fit : kBulkMaxStages;
+    const size_t smem = (size_t)kBulkWarps * ns * stage_bytes;
+    auto kern = k <= 8 ? combine_bulk_kernel<8> : combine_bulk_kernel<16>;
+    int per_sm = 1;
+    const cudaError_t err =
+        blocks_per_sm(reinterpret_cast<const void*>(kern), kBulkWarps * 32, smem, &per_sm);
+    if (err != cudaSuccess) return err;
+    return launch_pdl(env, kern, dim3((unsigned)(env.num_sms * per_sm)), dim3(kBulkWarps * 32),
+                      smem, ys, dst_pos, gates, sh, rs, T, H, k, N, o, hdr, ns, stage_bytes);
+  }
   // Capacity mode drops most slots of a skewed batch: then each task moves
   // little and its latency dominates, so wider slices with the next task's
   // metadata prefetched win; dense layouts do better with more warps.

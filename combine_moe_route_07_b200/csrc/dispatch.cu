@@ -344,9 +344,8 @@ __global__ void __launch_bounds__(kBulkWarps * 32)
 
 template <typename K>
 int grid_for(K kernel, const LaunchEnv& env, int64_t units) {
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess ||
-      per_sm < 1)
+  int per_sm = 1;
+  if (blocks_per_sm(reinterpret_cast<const void*>(kernel), kThreads, 0, &per_sm) != cudaSuccess)
     per_sm = 1;
   const int64_t need = (units + kThreads - 1) / kThreads;
   const int64_t cap = (int64_t)env.num_sms * per_sm;
@@ -379,14 +378,11 @@ cudaError_t launch_dispatch_bf16(const LaunchEnv& env, const void* x, const int3
     if (stages > kBulkMaxStages) stages = kBulkMaxStages;
     if (stages >= 2) {
       const size_t smem = (size_t)kBulkWarps * stages * stage_bytes;
-      cudaError_t err = cudaFuncSetAttribute(dispatch_bf16_bulk_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      int per_sm = 1;
+      const cudaError_t err =
+          blocks_per_sm(reinterpret_cast<const void*>(dispatch_bf16_bulk_kernel),
+                        kBulkWarps * 32, smem, &per_sm);
       if (err != cudaSuccess) return err;
-      int per_sm = 0;
-      err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dispatch_bf16_bulk_kernel,
-                                                          kBulkWarps * 32, smem);
-      if (err != cudaSuccess) return err;
-      if (per_sm < 1) per_sm = 1;
       int64_t grid = (int64_t)per_sm * env.num_sms;
       const int64_t need = ((int64_t)T * nsl + kBulkWarps - 1) / kBulkWarps;
       if (grid > need) grid = need;
@@ -421,14 +417,10 @@ cudaError_t launch_dispatch_fp8(const LaunchEnv& env, const void* x, const int32
       (reinterpret_cast<uintptr_t>(out) & 15u) == 0) {
     const uint32_t stage_bytes = (uint32_t)(((size_t)H + H / 32 + 127) / 128 * 128);
     const size_t smem = (size_t)kBulkWarps * kFp8Stages * stage_bytes;
-    cudaError_t err = cudaFuncSetAttribute(dispatch_fp8_bulk_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int per_sm = 1;
+    const cudaError_t err = blocks_per_sm(reinterpret_cast<const void*>(dispatch_fp8_bulk_kernel),
+                                          kBulkWarps * 32, smem, &per_sm);
     if (err != cudaSuccess) return err;
-    int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dispatch_fp8_bulk_kernel,
-                                                        kBulkWarps * 32, smem);
-    if (err != cudaSuccess) return err;
-    if (per_sm < 1) per_sm = 1;
     int64_t grid = (int64_t)per_sm * env.num_sms;
     const int64_t need = ((int64_t)T + kBulkWarps - 1) / kBulkWarps;
     if (grid > need) grid = need;

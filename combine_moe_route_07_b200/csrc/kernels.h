@@ -33,6 +33,15 @@ cudaError_t launch_pdl(const LaunchEnv& env, void (*kernel)(KArgs...), dim3 grid
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// Resident CTAs per SM (at least 1) of `kernel` at this block size and
+// dynamic shared memory on the current device, after raising the kernel's
+// dynamic shared-memory limit to at least `smem` (when smem > 0).  Every
+// launch of a kernel with dynamic shared memory above 48 KiB less its static
+// shared memory must come through here first.  Both
+// are cached per (device, kernel, threads, smem): the runtime's occupancy
+// query costs host time that would otherwise be paid on every launch.
+cudaError_t blocks_per_sm(const void* kernel, int threads, size_t smem, int* out);
+
 // Layout tiles: runs of TT consecutive tokens, TT a multiple of
 // kLayoutTileQuantum, at most kLayoutMaxTiles of them.  The workspace holds
 // two tables (used on alternate calls) of one row of E counters per tile.

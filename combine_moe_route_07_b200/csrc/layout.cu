@@ -387,10 +387,9 @@ cudaError_t launch_layout(const LaunchEnv& env, const int32_t* ids, int T, int E
   cudaError_t err;
   if (count_ids && T > 0) {
     const size_t smem = (size_t)E * sizeof(int32_t);
-    int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, count_kernel, kCountThreads, smem);
+    int per_sm = 1;
+    err = blocks_per_sm(reinterpret_cast<const void*>(count_kernel), kCountThreads, smem, &per_sm);
     if (err != cudaSuccess) return err;
-    if (per_sm < 1) per_sm = 1;
     int64_t blocks = ((int64_t)T + kLayoutTileQuantum - 1) / kLayoutTileQuantum;
     const int64_t cap = (int64_t)per_sm * env.num_sms;
     if (blocks > cap) blocks = cap;
@@ -421,11 +420,9 @@ cudaError_t launch_layout(const LaunchEnv& env, const int32_t* ids, int T, int E
   const int64_t entries = (int64_t)geom.TT * k;
   P.staged = entries <= kMaxStaged ? 1 : 0;
   const size_t smem = place_smem_words(E, P.staged ? (int)entries : 0) * sizeof(int32_t);
-  if (smem > 48 * 1024) {
-    err = cudaFuncSetAttribute(place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem);
-    if (err != cudaSuccess) return err;
-  }
+  int per_sm = 1;  // (raises the kernel's dynamic shared-memory limit to smem)
+  err = blocks_per_sm(reinterpret_cast<const void*>(place_kernel), kPlaceThreads, smem, &per_sm);
+  if (err != cudaSuccess) return err;
   return launch_pdl(env, place_kernel, dim3((unsigned)geom.G), dim3(kPlaceThreads), smem, P);
 }
 

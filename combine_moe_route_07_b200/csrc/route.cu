@@ -71,10 +71,9 @@ cudaError_t launch_nk(const LaunchEnv& env, const float* logits, const float* bi
                       uint32_t* tables, int TT, size_t table_words) {
   auto kern = route_kernel<NK, HIST>;
   const size_t smem = HIST ? (size_t)E * sizeof(int32_t) : 0;
-  int per_sm = 0;
-  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+  int per_sm = 1;
+  const cudaError_t err = blocks_per_sm(reinterpret_cast<const void*>(kern), kThreads, smem, &per_sm);
   if (err != cudaSuccess) return err;
-  if (per_sm < 1) per_sm = 1;
   int64_t blocks = ((int64_t)T + kWarps - 1) / kWarps;
   const int64_t cap = (int64_t)per_sm * env.num_sms;
   if (blocks > cap) blocks = cap;
