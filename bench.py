@@ -55,7 +55,7 @@ def parse():
 # ------------------------------------------------------------ byte counts --
 
 def algorithmic_bytes(w, kept_rows):
-    """Bytes each step must move (SURVEY's per-token figures, summed over the
+    """Bytes each step must move (the per-token figures of each step, summed over the
     rows actually kept)."""
     T, H, E, k = w.T, w.H, w.E, w.k
     row = 2 * H
@@ -465,6 +465,33 @@ def main():
     mean = [v / K_ops for v in sums]
     del g_probe
 
+    # dispatch and combine each on its own: a 256 MiB L2 write + read-back
+    # before every launch (outside the events, so dirty lines of the previous
+    # op are written back there), median over the iterations
+    iso_buf = flush_buf if flush_buf is not None else torch.empty(256 << 20, dtype=torch.uint8,
+                                                                  device=dev)
+    iso = {}
+    for name in ("dispatch", "combine"):
+        op = ops_probe[names_probe.index(name)]
+        g_op = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_op):
+            op()
+        times = []
+        for i in range(K_ops):
+            iso_buf.fill_(1)
+            iso_buf.view(torch.int64).sum()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g_op.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        del g_op
+        iso[name] = sorted(times)[len(times) // 2]
+    iso_n = K_ops
+    del iso_buf
+
     # end to end through the public API: pinned host inputs in, result out
     e2e = None
     if args.e2e_steps > 0:
@@ -532,7 +559,24 @@ def main():
         "dispatch_combine": {"tokens_per_s": world * T / (dc_ms * 1e-3),
                              "us": round(dc_ms * 1e3, 2), "gbs": round(dc_gbs, 1),
                              "frac": round(dc_gbs / peak, 4),
-                             "frac_of_8tbs": round(dc_gbs / 8000.0, 4)},
+                             "frac_of_8tbs": round(dc_gbs / 8000.0, 4),
+                             "method": (f"in the step: a replay of the step with event records "
+                                        f"between its kernels (no launch overlap across them), "
+                                        f"mean of {K_ops}")},
+        "dispatch_combine_isolated": {
+            "tokens_per_s": world * T / ((iso["dispatch"] + iso["combine"]) * 1e-3),
+            "us": round((iso["dispatch"] + iso["combine"]) * 1e3, 2),
+            "dispatch_us": round(iso["dispatch"] * 1e3, 2),
+            "combine_us": round(iso["combine"] * 1e3, 2),
+            "gbs": round((byts["dispatch"] + byts["combine"])
+                         / ((iso["dispatch"] + iso["combine"]) * 1e-3) / 1e9, 1),
+            "frac": round((byts["dispatch"] + byts["combine"])
+                          / ((iso["dispatch"] + iso["combine"]) * 1e-3) / 1e9 / peak, 4),
+            "frac_of_8tbs": round((byts["dispatch"] + byts["combine"])
+                                  / ((iso["dispatch"] + iso["combine"]) * 1e-3) / 1e9 / 8000.0,
+                                  4),
+            "method": (f"each op alone as a one-kernel CUDA graph, median of {iso_n}, "
+                       "256 MiB L2 write + read-back before each launch outside the events")},
         "kernels": kern,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(dom_gbs, 1),
                      "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",

@@ -54,7 +54,7 @@ typedef struct CUstream_st* moe_stream_t;
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1,    /* host check failed; nothing launched */
-  MOE_ERR_UNSUPPORTED = 2,    /* valid request outside what this build covers */
+  MOE_ERR_UNSUPPORTED = 2,    /* valid request outside what this library supports */
   MOE_ERR_WORKSPACE = 3,      /* workspace NULL, misaligned or too small */
   MOE_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
   MOE_ERR_DEVICE_RANGE = 5,   /* device: expert id or row index out of range */
