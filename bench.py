@@ -46,6 +46,9 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=200)
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--tokens", type=int, default=0,
+                   help="override the workload's token count (smaller cases for profiler "
+                        "captures; a changed workload, not a bench line)")
     p.add_argument("--path", choices=["fused3", "fused", "separate"], default="fused3",
                    help="steps 1-4 in one moe_route_layout_dispatch call; route+layout in one "
                         "moe_route_layout call; or one call per step")
@@ -281,6 +284,8 @@ def main():
     args = parse()
     from combine_moe_route_07_b200.workloads import WORKLOADS
     w = WORKLOADS[args.workload]
+    if args.tokens > 0:
+        w = w.with_(name=f"{w.name}_t{args.tokens}", T=args.tokens)
     if args.impl == "reference":
         return run_reference(args, w)
 
