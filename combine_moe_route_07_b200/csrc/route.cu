@@ -1,8 +1,20 @@
 // route.cu -- step 1: one warp per token (see route_core.cuh).  With a tile
-// table the kernel also counts the routed ids per layout tile: each CTA's
-// shared-memory histogram of its 8 tokens is added into the table row of the
-// tile those tokens belong to (integer adds, so the counts do not depend on
-// the order the CTAs run in).  That table is the first half of moe_layout.
+// table the kernel also counts the routed ids per layout tile: each CTA
+// keeps a shared-memory histogram of the tokens it routed in the current tile
+// and adds it into that tile's table row when its tokens move on to the next
+// tile (integer adds, so the counts do not depend on the order the CTAs run
+// in).  That table is the first half of moe_layout.
+//
+// Each CTA routes a contiguous run of tokens (a multiple of 8 long), warp w
+// the tokens c0 + w, c0 + w + 8, ...; a group of 8 never straddles a tile
+// (tiles are multiples of 16 tokens), so the CTA's histogram is flushed at
+// most once per tile it touches rather than once per group.
+//
+// STAGE (many experts per token, rows of 16-byte multiples): each warp keeps
+// two shared-memory row buffers and prefetches the logits of its next token by
+// bulk copy (TMA) while it routes the current one, so the row's DRAM latency
+// overlaps the selection arithmetic.
+#include "bulk.cuh"
 #include "common.cuh"
 #include "kernels.h"
 #include "route_core.cuh"
@@ -12,56 +24,126 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;  // tokens per CTA step
+constexpr int kWarps = kThreads / 32;  // tokens per CTA group
+constexpr uint64_t kRowTimeoutNs = 1000000000ull;
 
-template <int NK, bool HIST>
+template <int NK, bool HIST, bool STAGE>
 __global__ void __launch_bounds__(kThreads)
     route_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E,
                  int k, int renorm, int32_t* __restrict__ ids, float* __restrict__ gates,
-                 WsHeader* hdr, uint32_t* __restrict__ tables, int TT, size_t table_words) {
-  extern __shared__ int32_t hist[];  // [E] (HIST)
+                 WsHeader* hdr, uint32_t* __restrict__ tables, int TT, size_t table_words,
+                 int per) {
+  // dynamic: [hist: E int32, padded to 16 B] (HIST), [rows: kWarps x 2 x E floats] (STAGE)
+  extern __shared__ __align__(16) unsigned char dyn[];
   __shared__ uint32_t cand_all[kWarps][NK >= 8 ? 3 * kMaxCand : 1];
+  __shared__ uint64_t bars[kWarps][2];
+  int32_t* hist = reinterpret_cast<int32_t*>(dyn);
+  const size_t hist_bytes = HIST ? (((size_t)E * 4 + 15) & ~(size_t)15) : 0;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  float* buf = reinterpret_cast<float*>(dyn + hist_bytes) + (size_t)w * 2 * E;
+  if (STAGE && lane == 0) {
+    mbar_init(&bars[w][0], 1);
+    mbar_init(&bars[w][1], 1);
+    mbar_fence_init();
+  }
+  __syncwarp();
   pdl_wait();  // logits (and the tile table) may come from the kernel launched before
   pdl_trigger();
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   float b[NK];
   load_bias<NK>(bias, E, lane, b);
+  const int c0 = (int)min((int64_t)blockIdx.x * per, (int64_t)T);
+  const int c1 = min(T, c0 + per);
+  const int n = (c1 - c0 + kWarps - 1) / kWarps;  // groups: the same for every warp
   uint32_t* tab = nullptr;
+  int cur_tile = 0;
   if constexpr (HIST) {
     const uint32_t epoch = *reinterpret_cast<volatile uint32_t*>(&hdr->epoch);
     tab = tables + (size_t)(epoch & 1u) * table_words;
     for (int e = threadIdx.x; e < E; e += kThreads) hist[e] = 0;
     __syncthreads();
+    cur_tile = c0 / TT;
   }
-  for (int g0 = blockIdx.x * kWarps; g0 < T; g0 += gridDim.x * kWarps) {
-    const int t = g0 + w;
-    if (t < T) {
-      int tok[1] = {t}, e[1];
-      float g[1];
-      int nan_tok;
-      if constexpr (NK >= 8)
-        nan_tok = route_token_thr<NK>(logits, t, T, b, E, k, renorm, lane, cand_all[w], e[0], g[0]);
-      else
-        nan_tok = route_tokens<NK, 1>(logits, tok, T, b, E, k, renorm, lane, e, g);
-      if (nan_tok >= 0 && lane == 0) report(hdr, MOE_ERR_DEVICE_NAN, nan_tok);
-      if (lane < k) {
-        ids[(size_t)t * k + lane] = e[0];
-        gates[(size_t)t * k + lane] = g[0];
-        if constexpr (HIST) atomicAdd(&hist[e[0]], 1);
+  auto flush = [&](int tile) {  // caller: __syncthreads() before and after
+    uint32_t* row = tab + (size_t)tile * E;
+    for (int e = threadIdx.x; e < E; e += kThreads) {
+      const int c = hist[e];
+      if (c != 0) {
+        atomicAdd(row + e, (uint32_t)c);
+        hist[e] = 0;
       }
     }
-    if constexpr (HIST) {  // the 8 tokens lie in one tile (TT is a multiple of 8)
-      __syncthreads();
-      uint32_t* row = tab + (size_t)(g0 / TT) * E;
-      for (int e = threadIdx.x; e < E; e += kThreads) {
-        const int c = hist[e];
-        if (c != 0) {
-          atomicAdd(row + e, (uint32_t)c);
-          hist[e] = 0;
+  };
+  // STAGE: buffer s of this warp holds token (c0 + w + 8*i) for i of parity s
+  uint32_t parity = 0, pending = 0;
+  bool alive = true;
+  auto issue = [&](int tok, int sb) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bars[w][sb], (uint32_t)E * 4u);
+      bulk_load(buf + (size_t)sb * E, logits + (size_t)tok * E, (uint32_t)E * 4u, &bars[w][sb]);
+    }
+    pending |= 1u << sb;
+  };
+  if (STAGE && c0 + w < c1) issue(c0 + w, 0);
+
+  for (int i = 0; i < n; ++i) {
+    const int g0 = c0 + kWarps * i;
+    if constexpr (HIST) {
+      const int tile = g0 / TT;
+      if (tile != cur_tile) {
+        __syncthreads();
+        flush(cur_tile);
+        __syncthreads();
+        cur_tile = tile;
+      }
+    }
+    const int t = g0 + w;
+    if (t < c1 && alive) {
+      int e1 = 0;
+      float g1 = 0.0f;
+      int nan_tok;
+      if constexpr (STAGE) {
+        const int sb = i & 1;
+        // the other buffer was last read for token i-1 (done: __syncwarp below)
+        if (t + kWarps < c1) issue(t + kWarps, sb ^ 1);
+        const bool ok = __all_sync(
+            kFull, mbar_wait_bounded(&bars[w][sb], (parity >> sb) & 1u, kRowTimeoutNs));
+        if (ok) {
+          parity ^= 1u << sb;
+          pending &= ~(1u << sb);
+          nan_tok = route_token_thr<NK, true>(logits, t, T, b, E, k, renorm, lane, cand_all[w],
+                                              e1, g1, buf + (size_t)sb * E);
+        } else {
+          if (lane == 0) report(hdr, MOE_ERR_DEVICE_TIMEOUT, t);
+          alive = false;  // routes nothing more; still takes part in the CTA barriers
+        }
+      } else if constexpr (NK >= 8) {
+        nan_tok = route_token_thr<NK>(logits, t, T, b, E, k, renorm, lane, cand_all[w], e1, g1);
+      } else {
+        int tok[1] = {t}, ea[1];
+        float ga[1];
+        nan_tok = route_tokens<NK, 1>(logits, tok, T, b, E, k, renorm, lane, ea, ga);
+        e1 = ea[0];
+        g1 = ga[0];
+      }
+      if (alive) {
+        if (nan_tok >= 0 && lane == 0) report(hdr, MOE_ERR_DEVICE_NAN, nan_tok);
+        if (lane < k) {
+          ids[(size_t)t * k + lane] = e1;
+          gates[(size_t)t * k + lane] = g1;
+          if constexpr (HIST) atomicAdd(&hist[e1], 1);
         }
       }
-      __syncthreads();
     }
+    if constexpr (STAGE) __syncwarp();  // every lane is done with this buffer
+  }
+  if constexpr (STAGE) {  // copies still in flight land before the CTA exits
+    for (int sb = 0; sb < 2; ++sb)
+      if ((pending >> sb) & 1u)
+        (void)mbar_wait_bounded(&bars[w][sb], (parity >> sb) & 1u, kRowTimeoutNs);
+  }
+  if constexpr (HIST) {
+    __syncthreads();
+    if (n > 0) flush(cur_tile);
   }
 }
 
@@ -69,8 +151,11 @@ template <int NK, bool HIST>
 cudaError_t launch_nk(const LaunchEnv& env, const float* logits, const float* bias, int T, int E,
                       int k, int renorm, int32_t* ids, float* gates, WsHeader* hdr,
                       uint32_t* tables, int TT, size_t table_words) {
-  auto kern = route_kernel<NK, HIST>;
-  const size_t smem = HIST ? (size_t)E * sizeof(int32_t) : 0;
+  const size_t hist_bytes = HIST ? (((size_t)E * 4 + 15) & ~(size_t)15) : 0;
+  // rows staged by bulk copy: many keys per lane, 16-byte rows and base
+  const bool stage = NK >= 8 && (E % 4) == 0 && (reinterpret_cast<uintptr_t>(logits) & 15u) == 0;
+  auto kern = stage ? route_kernel<NK, HIST, NK >= 8> : route_kernel<NK, HIST, false>;
+  const size_t smem = hist_bytes + (stage ? (size_t)kWarps * 2 * E * sizeof(float) : 0);
   int per_sm = 1;
   const cudaError_t err = blocks_per_sm(reinterpret_cast<const void*>(kern), kThreads, smem, &per_sm);
   if (err != cudaSuccess) return err;
@@ -78,8 +163,14 @@ cudaError_t launch_nk(const LaunchEnv& env, const float* logits, const float* bi
   const int64_t cap = (int64_t)per_sm * env.num_sms;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
+  // contiguous runs of tokens, a multiple of kWarps long
+  int64_t per = ((int64_t)T + blocks - 1) / blocks;
+  per = (per + kWarps - 1) / kWarps * kWarps;
+  if (per < kWarps) per = kWarps;
+  blocks = ((int64_t)T + per - 1) / per;
+  if (blocks < 1) blocks = 1;
   return launch_pdl(env, kern, dim3((unsigned)blocks), dim3(kThreads), smem, logits, bias, T, E,
-                    k, renorm, ids, gates, hdr, tables, TT, table_words);
+                    k, renorm, ids, gates, hdr, tables, TT, table_words, (int)per);
 }
 
 template <bool HIST>

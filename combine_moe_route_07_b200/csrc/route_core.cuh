@@ -151,14 +151,16 @@ __device__ __forceinline__ int route_tokens(const float* __restrict__ logits, co
 // selected.  The warp compacts the keys >= tau (usually k to 2k of them) into
 // shared memory and runs the k selection rounds over at most two per lane.
 // More than kMaxCand candidates (heavy ties) falls back to route_tokens.
-// `cand` is this warp's 3*kMaxCand words of shared memory.
+// `cand` is this warp's 3*kMaxCand words of shared memory.  With SMEM the
+// token's logits are read from `srow` (a copy of the row in shared memory)
+// instead of from global memory.
 constexpr int kMaxCand = 64;
 
-template <int NK>
+template <int NK, bool SMEM = false>
 __device__ __forceinline__ int route_token_thr(const float* __restrict__ logits, int t, int T,
                                                const float (&b)[NK], int E, int k, int renorm,
                                                int lane, uint32_t* cand, int& sel_e,
-                                               float& gate) {
+                                               float& gate, const float* srow = nullptr) {
   float raw[NK];
   uint32_t code[NK];
   bool bad = false;
@@ -167,7 +169,7 @@ __device__ __forceinline__ int route_token_thr(const float* __restrict__ logits,
   for (int i = 0; i < NK; ++i) {
     const int e = lane + 32 * i;
     if (e < E) {
-      raw[i] = __ldcs(row + e);
+      raw[i] = SMEM ? srow[e] : __ldcs(row + e);
       const float key = __fadd_rn(raw[i], b[i]);
       bad |= (key != key);
       code[i] = order_code(key);
