@@ -85,6 +85,12 @@ __device__ __forceinline__ void bulk_store_hint(void* gmem_dst, const void* smem
                : "memory");
 }
 
+// An ordinary 4-byte store with an L2 cache policy.
+__device__ __forceinline__ void st_f32_hint(float* gmem, float v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(gmem), "f"(v), "l"(policy)
+               : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

@@ -267,21 +267,23 @@ __global__ void __launch_bounds__(kThreads)
 // codes: each warp streams its tokens; lane l quantises channels
 // 512g + 16l .. +16 of every 512-channel group g (a 128-channel block is 8
 // aligned lanes, its amax a 3-step xor shuffle), writes the codes and scales
-// into one of kFp8Stages shared-memory stages, and lane 0 issues the k bulk
-// stores of the codes row and of the scales row (one bulk group per token).
+// into one of kFp8Stages shared-memory stages; lane 0 issues the k bulk
+// stores of the codes row (one bulk group per token) and the lanes write the
+// k copies of the scales row with ordinary coalesced stores.
 constexpr int kFp8Stages = 4;
 
 __global__ void __launch_bounds__(kBulkWarps * 32)
     dispatch_fp8_bulk_kernel(const char* __restrict__ x, const int32_t* __restrict__ dst_pos,
                              int T, int H, int k, int64_t N, uint8_t* __restrict__ out,
-                             float* __restrict__ scales, uint32_t stage_bytes, WsHeader* hdr) {
+                             float* __restrict__ scales, uint32_t stage_bytes, int evict_first,
+                             WsHeader* hdr) {
   extern __shared__ __align__(128) unsigned char sbuf[];
   pdl_wait();  // x and dst_pos may come from the kernel launched just before
   pdl_trigger();
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t pol = l2_evict_first_policy();
   unsigned char* st = sbuf + (size_t)w * kFp8Stages * stage_bytes;
   const int groups = H >> 9;  // 512-channel groups
-  const uint32_t srow = (uint32_t)H >> 5;  // bytes of one scales row (H/128 floats)
   const size_t xrow = (size_t)H * 2;
   const int64_t stride = (int64_t)gridDim.x * kBulkWarps;
   int64_t t = (int64_t)blockIdx.x * kBulkWarps + w;
@@ -326,15 +328,28 @@ __global__ void __launch_bounds__(kBulkWarps * 32)
     }
     fence_proxy_async_smem();  // these shared-memory writes before the bulk stores
     __syncwarp();
+    // the scales row (H/128 floats, at most 64) by plain coalesced stores: a
+    // bulk copy per 64-byte row would cost the copy engine as much as a row
+    // of codes
+    const int nb = H >> 7;
+    const float s0 = lane < nb ? *reinterpret_cast<const float*>(sp + H + 4 * lane) : 0.0f;
+    const float s1 = lane + 32 < nb ? *reinterpret_cast<const float*>(sp + H + 4 * (lane + 32)) : 0.0f;
     for (int j = 0; j < k; ++j) {
       const int p = __shfl_sync(kFull, p_cur, j);
-      if (lane == 0 && p >= 0) {
-        if (p < N) {
-          bulk_store(out + (size_t)p * H, sp, (uint32_t)H);
-          bulk_store(reinterpret_cast<unsigned char*>(scales) + (size_t)p * srow, sp + H, srow);
-        } else {
-          report(hdr, MOE_ERR_DEVICE_RANGE, p);
-        }
+      if (p < 0) continue;
+      if (p >= N) {
+        if (lane == 0) report(hdr, MOE_ERR_DEVICE_RANGE, p);
+        continue;
+      }
+      float* srow_p = scales + (size_t)p * nb;
+      if (evict_first) {  // output larger than L2: its lines go back to DRAM early
+        if (lane == 0) bulk_store_hint(out + (size_t)p * H, sp, (uint32_t)H, pol);
+        if (lane < nb) st_f32_hint(srow_p + lane, s0, pol);
+        if (lane + 32 < nb) st_f32_hint(srow_p + lane + 32, s1, pol);
+      } else {
+        if (lane == 0) bulk_store(out + (size_t)p * H, sp, (uint32_t)H);
+        if (lane < nb) srow_p[lane] = s0;
+        if (lane + 32 < nb) srow_p[lane + 32] = s1;
       }
     }
     if (lane == 0) bulk_commit();
@@ -411,10 +426,9 @@ cudaError_t launch_dispatch_fp8(const LaunchEnv& env, const void* x, const int32
                                 WsHeader* hdr) {
   if (T == 0) return cudaSuccess;
   const int C8 = H / 8;
-  // bulk stores need 16-byte multiples: the scales row (H/32 bytes) asks for
-  // H % 512 == 0, and a 16-byte aligned scales buffer
-  if ((H % 512) == 0 && H <= 8192 && (reinterpret_cast<uintptr_t>(scales) & 15u) == 0 &&
-      (reinterpret_cast<uintptr_t>(out) & 15u) == 0) {
+  // staged variant: 512-channel groups per lane mapping (H % 512 == 0), a
+  // 16-byte aligned output for the row bulk stores, and at most 64 scales a row
+  if ((H % 512) == 0 && H <= 8192 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0) {
     const uint32_t stage_bytes = (uint32_t)(((size_t)H + H / 32 + 127) / 128 * 128);
     const size_t smem = (size_t)kBulkWarps * kFp8Stages * stage_bytes;
     int per_sm = 1;
@@ -424,9 +438,10 @@ cudaError_t launch_dispatch_fp8(const LaunchEnv& env, const void* x, const int32
     int64_t grid = (int64_t)per_sm * env.num_sms;
     const int64_t need = ((int64_t)T + kBulkWarps - 1) / kBulkWarps;
     if (grid > need) grid = need;
+    const int evict_first = ((int64_t)T * k * (H + H / 32) > (int64_t)192 << 20) ? 1 : 0;
     return launch_pdl(env, dispatch_fp8_bulk_kernel, dim3((unsigned)grid), dim3(kBulkWarps * 32),
                       smem, static_cast<const char*>(x), dst_pos, T, H, k, N,
-                      static_cast<uint8_t*>(out), scales, stage_bytes, hdr);
+                      static_cast<uint8_t*>(out), scales, stage_bytes, evict_first, hdr);
   }
   auto kern = dispatch_fp8_kernel<1>;
   const int grid = grid_for(kern, env, (int64_t)T * ((C8 + 31) / 32) * 32);
