@@ -34,6 +34,11 @@ def lib():
         L.orc_layout_rows.restype = i64
         L.orc_layout.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
         L.orc_layout.restype = i32
+        L.orc_layout_src_rows.argtypes = [i32, i32, i32, i32, i32, i32]
+        L.orc_layout_src_rows.restype = i64
+        L.orc_layout_src.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp,
+                                     vp]
+        L.orc_layout_src.restype = i32
         L.orc_dispatch_bf16.argtypes = [i32, i32, i32, vp, vp, vp]
         L.orc_dispatch_bf16.restype = None
         L.orc_quantize_row_fp8.argtypes = [i32, vp, vp, vp]
@@ -101,6 +106,34 @@ def layout(ids, E, R, capacity=0, align=1):
                           _p(out["dst_pos"]), _p(out["src_idx"]))
     if rc:
         raise OracleError(f"orc_layout status {rc}")
+    return out
+
+
+def layout_src_rows(T, E, k, R, capacity=0, align=1):
+    return int(lib().orc_layout_src_rows(T, E, k, R, capacity, align))
+
+
+def layout_src(ids, E, R, capacity=0, align=1):
+    """Per-source-rank layout (rows ordered by destination rank, source shard,
+    expert, token).  Returns dict(src_counts [R,E], seg_off [R*E+1],
+    pair_counts [R_src,R_dst], rank_off, rank_counts, dst_pos, src_idx)."""
+    ids = _c(ids, np.int32)
+    T, k = ids.shape
+    N = layout_src_rows(T, E, k, R, capacity, align)
+    out = dict(
+        src_counts=np.empty((R, E), np.int32),
+        seg_off=np.empty(R * E + 1, np.int32),
+        pair_counts=np.empty((R, R), np.int32),
+        rank_off=np.empty(R + 1, np.int32),
+        rank_counts=np.empty(R, np.int32),
+        dst_pos=np.empty((T, k), np.int32),
+        src_idx=np.empty(N, np.int32),
+    )
+    rc = lib().orc_layout_src(T, E, k, R, capacity, align, _p(ids), _p(out["src_counts"]),
+                              _p(out["seg_off"]), _p(out["pair_counts"]), _p(out["rank_off"]),
+                              _p(out["rank_counts"]), _p(out["dst_pos"]), _p(out["src_idx"]))
+    if rc:
+        raise OracleError(f"orc_layout_src status {rc}")
     return out
 
 

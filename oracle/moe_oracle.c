@@ -34,6 +34,9 @@
  *          activations feed a matmul that would cast them anyway.
  *   [OWN]  "Mixture-of-experts acceleration through overlap" (thecoregrid):
  *          remote-owner-aligned layout, every tile bound to one destination.
+ *   [MSG]  "GPU MoE all-to-all", section "The message-size distribution is
+ *          the whole story": an all-to-all over a group of ranks is one
+ *          logical message per (sender, receiver) pair, whatever the batch.
  *   [OCP]  OCP 8-bit Floating Point Specification (OFP8), E4M3 format:
  *          exponent bias 7, 3 mantissa bits, no infinities, S.1111.111 is
  *          NaN, largest finite magnitude 448, smallest subnormal 2^-9.
@@ -277,6 +280,104 @@ int orc_layout(int T, int E, int k, int R, int capacity, int align, const int32_
         continue;
       }
       int32_t p = expert_off[e] + c;
+      dst_pos[i] = p;
+      src_idx[p] = (int32_t)i;
+    }
+  }
+  free(cursor);
+  return ORC_OK;
+}
+
+/* Per-source-rank layout: the metadata and receive buffers a ragged
+ * all-to-all posts.  [TWO], [MSG], [RAG], [OWN]
+ *
+ * The T tokens are split into R source shards of Ts = ceil(T/R) consecutive
+ * tokens (shard s holds tokens s*Ts .. s*Ts+Ts-1; trailing shards may be short
+ * or empty).  Expert e lives on rank r = e / (E/R) as before.  The rows are
+ * the receive side of the exchange: ordered by destination rank r, then
+ * source shard s, then expert e (all ascending), then token order; segment
+ * (r, s, e) holds the assignments from shard s to expert e.
+ *
+ *   src_counts[s*E + e]   assignments of shard s to expert e (before drops)
+ *   seg_off[i]            first row of segment i = (r*R + s)*(E/R) + (e - r*(E/R));
+ *                         dropless: round_up(src_counts, align) rows per segment;
+ *                         capacity: exactly C rows per segment (per-sender-
+ *                         expert slots); seg_off[R*E] = rows used
+ *   pair_counts[s*R + r]  rows kept from shard s for rank r (the message size)
+ *   rank_off[r]           = seg_off[r*R*(E/R)] (rank r's slice); rank_off[R] = seg_off[R*E]
+ *   rank_counts[r]        rows kept for rank r from all shards
+ *   dst_pos, src_idx      as in orc_layout; capacity keeps the first C
+ *                         assignments of each (shard, expert) in token order
+ */
+int64_t orc_layout_src_rows(int T, int E, int k, int R, int capacity, int align) {
+  if (capacity > 0) return (int64_t)R * E * capacity;
+  return (int64_t)T * k + (int64_t)R * E * (align - 1);
+}
+
+int orc_layout_src(int T, int E, int k, int R, int capacity, int align, const int32_t* ids,
+                   int32_t* src_counts, int32_t* seg_off, int32_t* pair_counts,
+                   int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
+                   int32_t* src_idx) {
+  if (T < 0 || E < 1 || k < 1 || k > E || R < 1 || E % R != 0 || capacity < 0 || align < 1)
+    return ORC_BAD_ARG;
+  for (size_t i = 0; i < (size_t)T * k; ++i)
+    if (ids[i] < 0 || ids[i] >= E) return ORC_BAD_ID;
+  const int64_t N = orc_layout_src_rows(T, E, k, R, capacity, align);
+  const int Er = E / R;
+  const int Ts = T > 0 ? (T + R - 1) / R : 1;
+
+  /* counts per (source shard, expert) */
+  for (int s = 0; s < R; ++s)
+    for (int e = 0; e < E; ++e) src_counts[s * E + e] = 0;
+  for (int t = 0; t < T; ++t)
+    for (int j = 0; j < k; ++j) src_counts[(t / Ts) * E + ids[(size_t)t * k + j]] += 1;
+
+  /* segments in (rank, shard, expert) order; exclusive scan of their sizes */
+  int32_t run = 0;
+  for (int r = 0; r < R; ++r)
+    for (int s = 0; s < R; ++s)
+      for (int el = 0; el < Er; ++el) {
+        const int e = r * Er + el;
+        const int32_t c = src_counts[s * E + e];
+        seg_off[(r * R + s) * Er + el] = run;
+        run += capacity > 0 ? capacity : ((c + align - 1) / align) * align;
+      }
+  seg_off[R * E] = run;
+
+  /* message sizes and rank slices */
+  for (int s = 0; s < R; ++s)
+    for (int r = 0; r < R; ++r) {
+      int32_t kept = 0;
+      for (int e = r * Er; e < (r + 1) * Er; ++e) {
+        const int32_t c = src_counts[s * E + e];
+        kept += (capacity > 0 && c > capacity) ? capacity : c;
+      }
+      pair_counts[s * R + r] = kept;
+    }
+  for (int r = 0; r < R; ++r) {
+    rank_off[r] = seg_off[r * R * Er];
+    int32_t kept = 0;
+    for (int s = 0; s < R; ++s) kept += pair_counts[s * R + r];
+    rank_counts[r] = kept;
+  }
+  rank_off[R] = seg_off[R * E];
+
+  /* positions: token order, one cursor per (shard, expert) */
+  for (int64_t p = 0; p < N; ++p) src_idx[p] = -1;
+  int32_t* cursor = (int32_t*)calloc((size_t)R * E, sizeof(int32_t));
+  if (!cursor) return ORC_BAD_ARG;
+  for (int t = 0; t < T; ++t) {
+    const int s = t / Ts;
+    for (int j = 0; j < k; ++j) {
+      const size_t i = (size_t)t * k + j;
+      const int e = ids[i];
+      const int r = e / Er;
+      const int32_t c = cursor[s * E + e]++;
+      if (capacity > 0 && c >= capacity) {
+        dst_pos[i] = -1;
+        continue;
+      }
+      const int32_t p = seg_off[(r * R + s) * Er + (e - r * Er)] + c;
       dst_pos[i] = p;
       src_idx[p] = (int32_t)i;
     }
