@@ -24,9 +24,10 @@ from typing import Optional
 import torch
 
 from . import _binding
-from ._binding import MoeError, MOE_F_FP8, MOE_F_RENORM
+from ._binding import MoeError, MOE_F_FP8, MOE_F_RENORM, MOE_F_SRC_LAYOUT
 
-__all__ = ["MoeShape", "Workspace", "Layout", "MoeError", "moe_route", "moe_layout",
+__all__ = ["MoeShape", "Workspace", "Layout", "LayoutSrc", "MoeError", "moe_route", "moe_layout",
+           "moe_layout_src",
            "moe_route_layout", "moe_route_layout_dispatch",
            "moe_dispatch", "moe_combine", "moe_get_device_error", "moe_check",
            "moe_layout_rows", "moe_workspace_bytes"]
@@ -43,10 +44,12 @@ class MoeShape:
     align: int = 1
     renorm: bool = True
     fp8: bool = False
+    src_layout: bool = False  # rows follow the per-source-rank layout (moe_layout_src)
 
     @property
     def flags(self) -> int:
-        return (MOE_F_RENORM if self.renorm else 0) | (MOE_F_FP8 if self.fp8 else 0)
+        return ((MOE_F_RENORM if self.renorm else 0) | (MOE_F_FP8 if self.fp8 else 0)
+                | (MOE_F_SRC_LAYOUT if self.src_layout else 0))
 
     def c(self) -> _binding.MoeShapeC:
         return _binding.MoeShapeC(self.tokens, self.hidden, self.experts, self.k, self.ranks,
@@ -156,6 +159,42 @@ def moe_layout(shape: MoeShape, ids: torch.Tensor, *, ws: Workspace,
         _ptr(out.dst_pos, "dst_pos", torch.int32, (T, k)),
         _ptr(out.src_idx, "src_idx", torch.int32, (N,)), ws.ptr, ws.nbytes, _stream(dev))
     _check(st, "moe_layout")
+    return out
+
+
+@dataclasses.dataclass
+class LayoutSrc:
+    src_counts: torch.Tensor   # int32 [R,E]   per (source shard, expert)
+    seg_off: torch.Tensor      # int32 [R*E+1] segments in (rank, shard, expert) order
+    pair_counts: torch.Tensor  # int32 [R,R]   [source shard][destination rank]
+    rank_off: torch.Tensor     # int32 [R+1]
+    rank_counts: torch.Tensor  # int32 [R]
+    dst_pos: torch.Tensor      # int32 [T,k]
+    src_idx: torch.Tensor      # int32 [N]
+
+
+def moe_layout_src(shape: MoeShape, ids: torch.Tensor, *, ws: Workspace,
+                   out: Optional[LayoutSrc] = None) -> LayoutSrc:
+    """Per-source-rank layout (shape.src_layout must be set)."""
+    T, E, k, R = shape.tokens, shape.experts, shape.k, shape.ranks
+    N = shape.rows
+    dev = ids.device
+    if out is None:
+        i32 = dict(dtype=torch.int32, device=dev)
+        out = LayoutSrc(torch.empty((R, E), **i32), torch.empty(R * E + 1, **i32),
+                        torch.empty((R, R), **i32), torch.empty(R + 1, **i32),
+                        torch.empty(R, **i32), torch.empty((T, k), **i32),
+                        torch.empty(N, **i32))
+    st = _binding.lib().moe_layout_src(
+        ctypes.byref(shape.c()), _ptr(ids, "ids", torch.int32, (T, k)),
+        _ptr(out.src_counts, "src_counts", torch.int32, (R, E)),
+        _ptr(out.seg_off, "seg_off", torch.int32, (R * E + 1,)),
+        _ptr(out.pair_counts, "pair_counts", torch.int32, (R, R)),
+        _ptr(out.rank_off, "rank_off", torch.int32, (R + 1,)),
+        _ptr(out.rank_counts, "rank_counts", torch.int32, (R,)),
+        _ptr(out.dst_pos, "dst_pos", torch.int32, (T, k)),
+        _ptr(out.src_idx, "src_idx", torch.int32, (N,)), ws.ptr, ws.nbytes, _stream(dev))
+    _check(st, "moe_layout_src")
     return out
 
 

@@ -22,13 +22,14 @@ MOE_ERR_DEVICE_NAN = 7
 
 MOE_F_RENORM = 0x1
 MOE_F_FP8 = 0x2
+MOE_F_SRC_LAYOUT = 0x4
 
 # Every extern "C" symbol of include/moe_route07.h.
 EXPORTS = (
     "moe_abi_version", "moe_status_string", "moe_layout_rows", "moe_workspace_bytes",
     "moe_workspace_init", "moe_route", "moe_layout", "moe_dispatch", "moe_combine",
     "moe_get_device_error", "moe_layout_noalloc", "moe_route_layout",
-    "moe_route_layout_dispatch",
+    "moe_route_layout_dispatch", "moe_layout_src",
 )
 
 
@@ -82,6 +83,8 @@ def lib(path: str = None):
     L.moe_dispatch.restype = i32
     L.moe_combine.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.moe_combine.restype = i32
+    L.moe_layout_src.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_layout_src.restype = i32
     L.moe_layout_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.moe_layout_noalloc.restype = i32
     L.moe_get_device_error.argtypes = [vp, ctypes.POINTER(i32), vp]

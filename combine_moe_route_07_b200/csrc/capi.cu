@@ -21,26 +21,35 @@ bool shape_ok(const moe_shape_t* s) {
   if (s == nullptr) return false;
   const int64_t T = s->tokens, H = s->hidden, E = s->experts, k = s->k, R = s->ranks;
   if (T < 0 || H < 8 || (H % 8) != 0) return false;
-  if ((s->flags & ~(MOE_F_RENORM | MOE_F_FP8)) != 0u) return false;
+  if ((s->flags & ~(MOE_F_RENORM | MOE_F_FP8 | MOE_F_SRC_LAYOUT)) != 0u) return false;
   if ((s->flags & MOE_F_FP8) && (H % 128) != 0) return false;
   if (E < 1 || E > 1024 || R < 1 || (E % R) != 0) return false;
   if (k < 1 || k > E || k > 32) return false;
   if (s->capacity < 0 || s->align < 1 || s->align > (1 << 20)) return false;
   if (s->capacity > 0 && s->align != 1) return false;
   if (T * k >= (int64_t(1) << 30)) return false;
-  const int64_t rows = s->capacity > 0 ? E * s->capacity : T * k + E * (s->align - 1);
+  const int64_t segs = (s->flags & MOE_F_SRC_LAYOUT) ? R * E : E;  // R*E <= 2^20
+  const int64_t rows = s->capacity > 0 ? segs * s->capacity : T * k + segs * (s->align - 1);
   if (rows >= (int64_t(1) << 31)) return false;
   if (T * (H / 8) >= (int64_t(1) << 31)) return false;
   return true;
 }
 
+bool src_layout(const moe_shape_t* s) { return (s->flags & MOE_F_SRC_LAYOUT) != 0u; }
+
 int64_t rows_of(const moe_shape_t* s) {
-  return s->capacity > 0 ? int64_t(s->experts) * s->capacity
-                         : int64_t(s->tokens) * s->k + int64_t(s->experts) * (s->align - 1);
+  const int64_t segs = src_layout(s) ? int64_t(s->ranks) * s->experts : int64_t(s->experts);
+  return s->capacity > 0 ? segs * s->capacity
+                         : int64_t(s->tokens) * s->k + segs * (s->align - 1);
 }
 
-// Workspace: header, then two tile tables of equal size (words a multiple of 4).
+// Workspace: header, then two tile tables of equal size (words a multiple of
+// 4); for the per-source-rank layout, header + part counts + kept prefix.
 size_t ws_bytes_of(const moe_shape_t* s) {
+  if (src_layout(s))
+    return kHeaderBytes + (moe::layout_src_part_words(s->tokens, s->experts, s->ranks) +
+                           moe::layout_src_cum_words(s->experts, s->ranks)) *
+                              sizeof(int32_t);
   const size_t words = (moe::layout_table_words(s->tokens, s->experts) + 3) / 4 * 4;
   return kHeaderBytes + 2 * words * sizeof(uint32_t);
 }
@@ -130,7 +139,7 @@ moe_status_t moe_layout(const moe_shape_t* shape, const int32_t* ids, int32_t* c
                         int32_t* expert_off, int32_t* rank_off, int32_t* rank_counts,
                         int32_t* dst_pos, int32_t* src_idx, void* ws, size_t ws_bytes,
                         moe_stream_t stream) {
-  if (!shape_ok(shape)) return MOE_ERR_INVALID_ARG;
+  if (!shape_ok(shape) || src_layout(shape)) return MOE_ERR_INVALID_ARG;
   const int64_t N = rows_of(shape);
   if (counts == nullptr || expert_off == nullptr || rank_off == nullptr ||
       rank_counts == nullptr)
@@ -150,11 +159,39 @@ moe_status_t moe_layout(const moe_shape_t* shape, const int32_t* ids, int32_t* c
                                       rank_off, rank_counts, dst_pos, src_idx, true));
 }
 
+moe_status_t moe_layout_src(const moe_shape_t* shape, const int32_t* ids, int32_t* src_counts,
+                            int32_t* seg_off, int32_t* pair_counts, int32_t* rank_off,
+                            int32_t* rank_counts, int32_t* dst_pos, int32_t* src_idx, void* ws,
+                            size_t ws_bytes, moe_stream_t stream) {
+  if (!shape_ok(shape) || !src_layout(shape)) return MOE_ERR_INVALID_ARG;
+  const int64_t N = rows_of(shape);
+  if (src_counts == nullptr || seg_off == nullptr || pair_counts == nullptr ||
+      rank_off == nullptr || rank_counts == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (shape->tokens > 0 && (ids == nullptr || dst_pos == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (N > 0 && src_idx == nullptr) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {ids, src_counts, seg_off, pair_counts, rank_off, rank_counts, dst_pos,
+                        src_idx};
+  for (const void* p : ptrs)
+    if (!aligned(p, 4)) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = ws_ok(shape, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  WsHeader* hdr = static_cast<WsHeader*>(ws);
+  int32_t* partc = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + kHeaderBytes);
+  int32_t* keptcum =
+      partc + moe::layout_src_part_words(shape->tokens, shape->experts, shape->ranks);
+  return from_cuda(moe::launch_layout_src(env_of(stream), ids, shape->tokens, shape->experts,
+                                          shape->k, shape->ranks, shape->capacity, shape->align,
+                                          N, partc, keptcum, hdr, src_counts, seg_off,
+                                          pair_counts, rank_off, rank_counts, dst_pos,
+                                          src_idx));
+}
+
 moe_status_t moe_route_layout(const moe_shape_t* shape, const float* logits, const float* bias,
                               int32_t* ids, float* gates, int32_t* counts, int32_t* expert_off,
                               int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
                               int32_t* src_idx, void* ws, size_t ws_bytes, moe_stream_t stream) {
-  if (!shape_ok(shape)) return MOE_ERR_INVALID_ARG;
+  if (!shape_ok(shape) || src_layout(shape)) return MOE_ERR_INVALID_ARG;
   const int64_t N = rows_of(shape);
   if (counts == nullptr || expert_off == nullptr || rank_off == nullptr ||
       rank_counts == nullptr)
@@ -191,7 +228,7 @@ moe_status_t moe_route_layout_dispatch(const moe_shape_t* shape, const float* lo
                                        int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
                                        int32_t* src_idx, void* out, float* scales, void* ws,
                                        size_t ws_bytes, moe_stream_t stream) {
-  if (!shape_ok(shape)) return MOE_ERR_INVALID_ARG;
+  if (!shape_ok(shape) || src_layout(shape)) return MOE_ERR_INVALID_ARG;
   const bool fp8 = (shape->flags & MOE_F_FP8) != 0u;
   if (shape->tokens > 0 && (x == nullptr || out == nullptr || (fp8 && scales == nullptr)))
     return MOE_ERR_INVALID_ARG;

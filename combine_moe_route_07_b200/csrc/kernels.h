@@ -70,6 +70,41 @@ inline size_t layout_table_words(int T, int E) {
   return (size_t)rows * (size_t)E;
 }
 
+// Per-source-rank layout geometry: R source shards of Ts consecutive tokens,
+// each cut into P parts of TP tokens (about 256 parts in all, at least 16
+// tokens each); one CTA per part counts and later places its assignments.
+struct SrcGeom {
+  int Ts;  // tokens per shard
+  int TP;  // tokens per part
+  int P;   // parts per shard
+};
+inline SrcGeom layout_src_geom(int T, int R) {
+  SrcGeom g;
+  g.Ts = T > 0 ? (T + R - 1) / R : 1;
+  int want = 256 / R;
+  if (want < 1) want = 1;
+  int tp = (g.Ts + want - 1) / want;
+  if (tp < 16) tp = 16;
+  g.TP = tp;
+  g.P = (g.Ts + tp - 1) / tp;
+  return g;
+}
+// Workspace words after the header: part counts [R][P][E], then the
+// exclusive prefix of kept rows over the R*E segments (+1).
+inline size_t layout_src_part_words(int T, int E, int R) {
+  const SrcGeom g = layout_src_geom(T, R);
+  return ((size_t)R * g.P * E + 3) / 4 * 4;
+}
+inline size_t layout_src_cum_words(int E, int R) { return ((size_t)R * E + 1 + 3) / 4 * 4; }
+
+// Per-source-rank layout: count parts, scan segments, place (three kernels
+// chained by PDL).  partc and keptcum are workspace scratch.
+cudaError_t launch_layout_src(const LaunchEnv& env, const int32_t* ids, int T, int E, int k, int R,
+                              int capacity, int align, int64_t N, int32_t* partc,
+                              int32_t* keptcum, WsHeader* hdr, int32_t* src_counts,
+                              int32_t* seg_off, int32_t* pair_counts, int32_t* rank_off,
+                              int32_t* rank_counts, int32_t* dst_pos, int32_t* src_idx);
+
 // tables != nullptr: also add each routed token's ids into the layout tile
 // table the next place pass reads (the fused route + layout path).  `tables`
 // holds two tables of `half_words` words each.

@@ -65,7 +65,7 @@ extern "C" moe_status_t moe_layout_noalloc(const moe_shape_t* shape, const int32
                                            moe_stream_t stream) {
   // Shape checks: the same limits as moe_layout, plus the static table size.
   const int64_t rows = moe_layout_rows(shape);
-  if (rows < 0) return MOE_ERR_INVALID_ARG;
+  if (rows < 0 || (shape->flags & MOE_F_SRC_LAYOUT) != 0u) return MOE_ERR_INVALID_ARG;
   const size_t need = moe_workspace_bytes(shape);
   if (need == 0) return MOE_ERR_INVALID_ARG;
   if (need > kMoeNoallocScratchBytes) return MOE_ERR_UNSUPPORTED;

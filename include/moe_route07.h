@@ -65,6 +65,7 @@ typedef enum {
 /* flags */
 #define MOE_F_RENORM 0x1u /* gates: softmax over the k selected experts (else over all E) */
 #define MOE_F_FP8 0x2u    /* dispatch writes e4m3 codes + per-128-channel fp32 scales */
+#define MOE_F_SRC_LAYOUT 0x4u /* rows follow the per-source-rank layout (moe_layout_src) */
 
 /* Problem description (host memory).
  *   tokens   T >= 0
@@ -86,9 +87,10 @@ typedef struct {
   uint32_t flags;
 } moe_shape_t;
 
-/* Rows N of the dispatched buffer: dropless T*k + E*(align-1), capacity E*C.
- * A static bound, so buffers are sized without reading counts back.
- * Returns -1 for an invalid shape. */
+/* Rows N of the dispatched buffer: dropless T*k + E*(align-1), capacity E*C;
+ * with MOE_F_SRC_LAYOUT dropless T*k + R*E*(align-1), capacity R*E*C.  A
+ * static bound, so buffers are sized without reading counts back.  Returns -1
+ * for an invalid shape. */
 int64_t moe_layout_rows(const moe_shape_t* shape);
 
 /* Bytes of device workspace the calls need for `shape` (error word, the
@@ -131,11 +133,45 @@ moe_status_t moe_route(const moe_shape_t* shape, const float* logits, const floa
  * Within an expert, rows follow token order; in capacity mode the first C
  * assignments in that order are kept.  Results are deterministic: no output
  * depends on block scheduling.  An id outside [0,E) sets
- * MOE_ERR_DEVICE_RANGE and that assignment is treated as dropped. */
+ * MOE_ERR_DEVICE_RANGE and that assignment is treated as dropped.  A shape
+ * with MOE_F_SRC_LAYOUT returns MOE_ERR_INVALID_ARG here and in the fused and
+ * allocation-free layout calls (use moe_layout_src). */
 moe_status_t moe_layout(const moe_shape_t* shape, const int32_t* ids, int32_t* counts,
                         int32_t* expert_off, int32_t* rank_off, int32_t* rank_counts,
                         int32_t* dst_pos, int32_t* src_idx, void* ws, size_t ws_bytes,
                         moe_stream_t stream);
+
+/* Per-source-rank layout: the metadata and receive-side rows of a ragged
+ * all-to-all ("GPU MoE all-to-all", sections "Two collectives per layer, and
+ * what each one moves" -- counts before payload -- and "The message-size
+ * distribution is the whole story" -- one message per (sender, receiver);
+ * "MoE All-to-All Dispatch and Ragged Routing", section "Fixed Capacity vs.
+ * Ragged Routing" -- per-sender-expert slots).  The shape must carry
+ * MOE_F_SRC_LAYOUT; no page gives this interface.
+ * The T tokens form R source shards of Ts = ceil(T/R) consecutive tokens
+ * (shard s = tokens s*Ts .. s*Ts+Ts-1; trailing shards may be short or
+ * empty).  Rows are ordered by destination rank r, then source shard s, then
+ * expert e of rank r, then token order; segment (r, s, e) has index
+ * i = (r*R + s)*(E/R) + e - r*(E/R) and holds round_up(count, align) rows
+ * (dropless) or exactly C rows (capacity: the first C assignments of shard s
+ * to expert e in token order are kept).
+ *   ids          int32 [T,k]     expert ids
+ *   src_counts   int32 [R,E]     assignments of shard s to expert e, before drops
+ *   seg_off      int32 [R*E+1]   first row of segment i; [R*E] = rows used
+ *   pair_counts  int32 [R,R]     [s][r] rows kept from shard s for rank r:
+ *                                the size of the (s -> r) message
+ *   rank_off     int32 [R+1]     first row of rank r's slice; [R] = rows used
+ *   rank_counts  int32 [R]       rows kept for rank r from all shards
+ *   dst_pos      int32 [T,k]     row of assignment (t,j); -1 if dropped
+ *   src_idx      int32 [N]       t*k+j in each row; -1 if the row is empty
+ * All caller-owned device buffers, 4-byte aligned.  The workspace is sized by
+ * moe_workspace_bytes of the same shape.  Deterministic; an id outside [0,E)
+ * sets MOE_ERR_DEVICE_RANGE and that assignment is dropped.  moe_dispatch
+ * and moe_combine take the resulting dst_pos with the same shape. */
+moe_status_t moe_layout_src(const moe_shape_t* shape, const int32_t* ids, int32_t* src_counts,
+                            int32_t* seg_off, int32_t* pair_counts, int32_t* rank_off,
+                            int32_t* rank_counts, int32_t* dst_pos, int32_t* src_idx, void* ws,
+                            size_t ws_bytes, moe_stream_t stream);
 
 /* Steps 1-3 in one launch: moe_route followed by moe_layout, fused so the
  * ids never leave the CTA that routed them before they are counted.  Same
