@@ -46,6 +46,10 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=200)
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--layout", choices=["expert", "src"], default="expert",
+                   help="expert: rows by expert; src: the per-source-rank layout (rows by "
+                        "destination rank, source shard, expert), route + layout_src + dispatch "
+                        "+ combine as separate calls")
     p.add_argument("--tokens", type=int, default=0,
                    help="override the workload's token count (smaller cases for profiler "
                         "captures; a changed workload, not a bench line)")
@@ -69,6 +73,9 @@ def algorithmic_bytes(w, kept_rows):
     b["dispatch"] = T * row + kept_rows * disp_row_out + T * k * 4
     b["combine"] = kept_rows * row + T * k * 8 + T * row \
         + (T * row if w.shared else 0) + (T * row if w.residual else 0)
+    # per-source-rank layout: ids in, dst_pos and src_idx out, the [R,E]
+    # counts, the R*E+1 segment offsets and the [R,R] message sizes out
+    b["layout_src"] = T * k * 4 * 2 + w.rows_src * 4 + (2 * w.R * E + 1 + w.R * w.R) * 4
     # fused route + layout: the ids stay in the CTA between the two steps
     b["route_layout"] = b["route"] + b["layout"] - T * k * 4
     b["route_layout_dispatch"] = b["route_layout"] + b["dispatch"] - T * k * 4
@@ -307,8 +314,10 @@ def main():
     from combine_moe_route_07_b200.workloads import make_inputs
 
     inp = make_inputs(w, seed=w.seed + rank)
+    src = args.layout == "src"
     shape = m.MoeShape(tokens=w.T, hidden=w.H, experts=w.E, k=w.k, ranks=w.R,
-                       capacity=w.capacity, align=w.align, renorm=w.renorm, fp8=w.fp8)
+                       capacity=w.capacity_src if src else w.capacity, align=w.align,
+                       renorm=w.renorm, fp8=w.fp8, src_layout=src)
     ws = m.Workspace(shape, dev)
     x = inp.x.to(dev)
     logits = inp.logits.to(dev)
@@ -317,9 +326,15 @@ def main():
     i32 = dict(dtype=torch.int32, device=dev)
     ids = torch.empty((T, k), **i32)
     gates = torch.empty((T, k), dtype=torch.float32, device=dev)
-    lay = m.Layout(torch.empty(w.E, **i32), torch.empty(w.E + 1, **i32),
-                   torch.empty(w.R + 1, **i32), torch.empty(w.R, **i32),
-                   torch.empty((T, k), **i32), torch.empty(N, **i32))
+    if src:
+        lay = m.LayoutSrc(torch.empty((w.R, w.E), **i32), torch.empty(w.R * w.E + 1, **i32),
+                          torch.empty((w.R, w.R), **i32), torch.empty(w.R + 1, **i32),
+                          torch.empty(w.R, **i32), torch.empty((T, k), **i32),
+                          torch.empty(N, **i32))
+    else:
+        lay = m.Layout(torch.empty(w.E, **i32), torch.empty(w.E + 1, **i32),
+                       torch.empty(w.R + 1, **i32), torch.empty(w.R, **i32),
+                       torch.empty((T, k), **i32), torch.empty(N, **i32))
     if w.fp8:
         xd = torch.empty((N, w.H), dtype=torch.float8_e4m3fn, device=dev)
         sc = torch.empty((N, w.H // 128), dtype=torch.float32, device=dev)
@@ -332,13 +347,21 @@ def main():
 
     def route_layout_dispatch():
         m.moe_route(shape, logits, bias, ws=ws, ids=ids, gates=gates)
-        m.moe_layout(shape, ids, ws=ws, out=lay)
+        if src:
+            m.moe_layout_src(shape, ids, ws=ws, out=lay)
+        else:
+            m.moe_layout(shape, ids, ws=ws, out=lay)
         m.moe_dispatch(shape, x, lay.dst_pos, ws=ws, out=xd, scales=sc)
 
     # the expert stand-in's output for this batch, prepared once
     route_layout_dispatch()
     if w.fp8:
         y = (xd.float() * sc.repeat_interleave(128, dim=1)).to(torch.bfloat16)
+    elif w.expert == "scale" and src:
+        e = ids.flatten()[lay.src_idx.clamp(min=0).long()].long()
+        s = (torch.arange(1, w.E + 1, dtype=torch.float32, device=dev)
+             / torch.tensor(float(w.E), device=dev))[e]
+        y = (xd.float() * s[:, None]).to(torch.bfloat16)
     elif w.expert == "scale":
         rows = torch.arange(N, device=dev, dtype=torch.int32)
         e = (torch.searchsorted(lay.expert_off, rows, right=True) - 1).clamp(min=0)
@@ -353,7 +376,7 @@ def main():
 
     L2_BYTES = 126 * 10**6
     _b = algorithmic_bytes(w, kept_rows)
-    touched = _b["route"] + _b["layout"] + _b["dispatch"] + _b["combine"]
+    touched = _b["route"] + _b["layout_src" if src else "layout"] + _b["dispatch"] + _b["combine"]
     flush_between = touched < 2 * L2_BYTES
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush_between else None
 
@@ -371,7 +394,16 @@ def main():
         lambda: m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared,
                               residual=residual, out=out),
     )
-    if args.path == "fused3":
+    if src:
+        names = ("route", "layout_src", "dispatch", "combine")
+        ops = (
+            lambda: m.moe_route(shape, logits, bias, ws=ws, ids=ids, gates=gates),
+            lambda: m.moe_layout_src(shape, ids, ws=ws, out=lay),
+            lambda: m.moe_dispatch(shape, x, lay.dst_pos, ws=ws, out=xd, scales=sc),
+            lambda: m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared,
+                                  residual=residual, out=out),
+        )
+    elif args.path == "fused3":
         names = ("route_layout_dispatch", "combine")
         ops = (
             lambda: m.moe_route_layout_dispatch(shape, logits, x, bias, ws=ws, ids=ids, gates=gates,
@@ -448,8 +480,8 @@ def main():
     # per-kernel breakdown: a probe graph of the same step with event-record
     # nodes between the kernels, replayed after an L2 flush and read back one
     # replay at a time
-    probe_names = names if args.path != "fused3" else names_probe
-    probe_ops = ops if args.path != "fused3" else ops_probe
+    probe_names = names if (src or args.path != "fused3") else names_probe
+    probe_ops = ops if (src or args.path != "fused3") else ops_probe
     n_ops = len(probe_ops)
     probe_ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ops + 1)]
     g_probe = torch.cuda.CUDAGraph()
@@ -554,12 +586,15 @@ def main():
         "dtype": "fp8-e4m3 dispatch, bf16 rows, fp32 accumulate" if w.fp8 else "bf16",
         "data": "synthetic",
         "config": {"workload": w.describe(), "tokens": T, "hidden": w.H, "experts": w.E,
-                   "k": k, "ranks": w.R, "capacity": w.capacity, "rows": N,
+                   "k": k, "ranks": w.R, "capacity": shape.capacity, "rows": N,
                    "kept_rows": kept_rows, "parallelism": f"replicas x{world}",
                    "l2": ("256 MiB write + read between timed steps, outside the step events"
                           if flush_between else
                           f"no flush: inputs larger than L2 ({touched / 1e6:.0f} MB touched per "
                           f"step vs 126 MB L2), steps back to back"),
+                   "layout": ("per-source-rank: rows by destination rank, source shard "
+                              "(R shards of ceil(T/R) tokens), expert, token") if src else
+                             "rows by expert, token",
                    "step": " + ".join(names) + ", one CUDA graph"},
         "dispatch_combine": {"tokens_per_s": world * T / (dc_ms * 1e-3),
                              "us": round(dc_ms * 1e3, 2), "gbs": round(dc_gbs, 1),
@@ -587,7 +622,7 @@ def main():
                      "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
                      "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
                      "traffic": ncu_traffic(dom, w.name)},
-        "gpu_launches": {"fused3": 4, "fused": 4, "separate": 5}[args.path] * K,
+        "gpu_launches": (7 if src else {"fused3": 4, "fused": 4, "separate": 5}[args.path]) * K,
         "clocks": clocks,
         "e2e": e2e,
     }

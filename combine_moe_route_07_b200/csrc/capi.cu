@@ -178,11 +178,11 @@ moe_status_t moe_layout_src(const moe_shape_t* shape, const int32_t* ids, int32_
   if (st != MOE_OK) return st;
   WsHeader* hdr = static_cast<WsHeader*>(ws);
   int32_t* partc = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + kHeaderBytes);
-  int32_t* keptcum =
+  int32_t* scratch =
       partc + moe::layout_src_part_words(shape->tokens, shape->experts, shape->ranks);
   return from_cuda(moe::launch_layout_src(env_of(stream), ids, shape->tokens, shape->experts,
                                           shape->k, shape->ranks, shape->capacity, shape->align,
-                                          N, partc, keptcum, hdr, src_counts, seg_off,
+                                          N, partc, scratch, hdr, src_counts, seg_off,
                                           pair_counts, rank_off, rank_counts, dst_pos,
                                           src_idx));
 }

@@ -90,18 +90,23 @@ inline SrcGeom layout_src_geom(int T, int R) {
   return g;
 }
 // Workspace words after the header: part counts [R][P][E], then the
-// exclusive prefix of kept rows over the R*E segments (+1).
+// per-segment totals [R*E], the exclusive prefix of kept rows over the R*E
+// segments (+1) and one 64-bit sum per chunk of 1024 segments.
 inline size_t layout_src_part_words(int T, int E, int R) {
   const SrcGeom g = layout_src_geom(T, R);
   return ((size_t)R * g.P * E + 3) / 4 * 4;
 }
-inline size_t layout_src_cum_words(int E, int R) { return ((size_t)R * E + 1 + 3) / 4 * 4; }
+inline size_t layout_src_cum_words(int E, int R) {
+  const size_t chunks = ((size_t)R * E + 1023) / 1024;
+  return ((size_t)R * E + 3) / 4 * 4 + ((size_t)R * E + 1 + 3) / 4 * 4 + (2 * chunks + 3) / 4 * 4;
+}
 
-// Per-source-rank layout: count parts, scan segments, place (three kernels
-// chained by PDL).  partc and keptcum are workspace scratch.
+// Per-source-rank layout: count parts, reduce, scan segments, place (four
+// kernels chained by PDL).  partc (layout_src_part_words) and scratch
+// (layout_src_cum_words) are workspace.
 cudaError_t launch_layout_src(const LaunchEnv& env, const int32_t* ids, int T, int E, int k, int R,
                               int capacity, int align, int64_t N, int32_t* partc,
-                              int32_t* keptcum, WsHeader* hdr, int32_t* src_counts,
+                              int32_t* scratch, WsHeader* hdr, int32_t* src_counts,
                               int32_t* seg_off, int32_t* pair_counts, int32_t* rank_off,
                               int32_t* rank_counts, int32_t* dst_pos, int32_t* src_idx);
 

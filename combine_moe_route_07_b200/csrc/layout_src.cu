@@ -15,15 +15,17 @@
 // align) rows, capacity segments exactly C rows (the first C assignments of
 // the pair in token order are kept).
 //
-// Three kernels, chained by programmatic dependent launch:
+// Four kernels, chained by programmatic dependent launch:
 //   part count  one CTA per part (a run of TP tokens inside one shard):
 //               shared-memory histogram, written whole to its workspace row
 //               (no atomics to global memory, nothing to clear);
-//   scan        one CTA: per-(shard, expert) totals, segment sizes and kept
-//               rows in (rank, shard, expert) order, one block scan per
-//               4096 segments with a running carry; message sizes per
-//               (shard, rank) and rank slices from the kept-row prefix;
-//   place       one CTA per part: rank offset of each expert from the
+//   reduce      one CTA per chunk of 1024 segments in (rank, shard, expert)
+//               order: per-segment totals from the part counts, and the
+//               chunk's sums of rows and kept rows;
+//   scan        one CTA per chunk: the earlier chunks' sums, then a block
+//               scan of the chunk's segments (segment offsets, kept prefix);
+//   place       one CTA per part (all CTAs also write the message sizes per
+//               (shard, rank) and the rank slices): rank offset of each expert from the
 //               earlier parts of the same shard, then each warp ranks a
 //               contiguous run of assignments with __match_any_sync, warps
 //               are chained in token order through per-warp counters, and
@@ -38,8 +40,10 @@ namespace {
 
 constexpr int kSrcThreads = 256;
 constexpr int kSrcWarps = kSrcThreads / 32;
-constexpr int kScanThreads = 1024;
-constexpr int kScanPer = 4;  // segments per thread per scan chunk
+constexpr int kSegPerThread = 4;
+constexpr int kChunkSeg = kSrcThreads * kSegPerThread;  // segments per reduce/scan CTA
+static_assert(kChunkSeg == 1024, "layout_src_cum_words sizes the chunk sums for 1024 segments");
+constexpr int kRounds = 4;  // 32-assignment rounds whose ids are loaded together
 
 struct SrcParams {
   const int32_t* ids;
@@ -47,7 +51,9 @@ struct SrcParams {
   int Ts, TP, P;
   int64_t N;
   int32_t* partc;    // [R*P][E]
-  int32_t* keptcum;  // [R*E + 1]
+  int32_t* cnt;       // [R*E] per segment, in segment order
+  int32_t* keptcum;   // [R*E + 1]
+  int64_t* blocksum;  // [chunks] (rows << 32) | kept per chunk of kChunkSeg segments
   WsHeader* hdr;
   int32_t* src_counts;
   int32_t* seg_off;
@@ -87,10 +93,33 @@ __global__ void __launch_bounds__(kSrcThreads) src_count_kernel(const SrcParams 
   for (int e = threadIdx.x; e < P.E; e += kSrcThreads) row[e] = hist[e];
 }
 
-// Inclusive scan of a 64-bit value across the CTA (kScanThreads threads);
-// returns the inclusive prefix, and the CTA total in *total.
-__device__ int64_t scan_block64(int64_t v, int64_t* wsum, int64_t* total) {
-  constexpr int kW = kScanThreads / 32;
+// (rows << 32) | kept of one segment with `cnt` assignments
+__device__ __forceinline__ int64_t seg_value(const SrcParams& P, int cnt) {
+  const int C = P.capacity;
+  const int64_t rows = C > 0 ? C : (int64_t)((cnt + P.align - 1) / P.align) * P.align;
+  const int64_t kept = (C > 0 && cnt > C) ? C : cnt;
+  return (rows << 32) | kept;
+}
+
+// Sum of a 64-bit value over the CTA (kSrcThreads threads), to every thread.
+__device__ int64_t sum_block64(int64_t v, int64_t* wsum) {
+  constexpr int kW = kSrcThreads / 32;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  if (lane == 0) wsum[w] = v;
+  __syncthreads();
+  int64_t t = 0;
+#pragma unroll
+  for (int q = 0; q < kW; ++q) t += wsum[q];
+  __syncthreads();
+  return t;
+}
+
+// Exclusive scan of a 64-bit value over the CTA (kSrcThreads threads);
+// *total gets the CTA sum.
+__device__ int64_t excl_scan_block64(int64_t v, int64_t* wsum, int64_t* total) {
+  constexpr int kW = kSrcThreads / 32;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   int64_t x = v;
 #pragma unroll
@@ -100,80 +129,85 @@ __device__ int64_t scan_block64(int64_t v, int64_t* wsum, int64_t* total) {
   }
   if (lane == 31) wsum[w] = x;
   __syncthreads();
-  if (w == 0) {
-    int64_t s = lane < kW ? wsum[lane] : 0;
+  int64_t before = 0, all = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int64_t y = __shfl_up_sync(kFull, s, o);
-      if (lane >= o) s += y;
-    }
-    if (lane < kW) wsum[lane] = s;
+  for (int q = 0; q < kW; ++q) {
+    if (q < w) before += wsum[q];
+    all += wsum[q];
   }
   __syncthreads();
-  const int64_t r = x + (w > 0 ? wsum[w - 1] : 0);
-  *total = wsum[kW - 1];
-  __syncthreads();  // wsum is reused by the next call
-  return r;
+  *total = all;
+  return before + x - v;
 }
 
-__global__ void __launch_bounds__(kScanThreads) src_scan_kernel(const SrcParams P) {
-  __shared__ int64_t wsum[kScanThreads / 32];
+// segment i = (r*R + s)*Er + el  ->  expert e and shard s
+__device__ __forceinline__ void seg_coords(const SrcParams& P, int i, int& s, int& e) {
+  const int per_rank = P.R * P.Er;
+  const int r = i / per_rank;
+  const int rem = i - r * per_rank;
+  s = rem / P.Er;
+  e = r * P.Er + (rem - s * P.Er);
+}
+
+// One CTA per chunk of kChunkSeg segments in (rank, shard, expert) order:
+// per-segment totals from the part counts (also the caller's src_counts),
+// and the chunk's sum of (rows, kept).
+__global__ void __launch_bounds__(kSrcThreads) src_reduce_kernel(const SrcParams P) {
+  __shared__ int64_t wsum[kSrcWarps];
   pdl_wait();  // the part counts are complete
   pdl_trigger();
   const int nseg = P.R * P.E;
-  const int C = P.capacity;
-  const int per_rank = P.R * P.Er;  // segments of one destination rank (= E)
-  int64_t carry = 0;                // (rows << 32) | kept, summed so far
-  for (int c0 = 0; c0 < nseg; c0 += kScanThreads * kScanPer) {
-    int64_t v[kScanPer];
-    int64_t local = 0;
+  const int c0 = blockIdx.x * kChunkSeg;
+  int64_t local = 0;
 #pragma unroll
-    for (int u = 0; u < kScanPer; ++u) {
-      const int i = c0 + threadIdx.x * kScanPer + u;
-      v[u] = 0;
-      if (i < nseg) {
-        const int r = i / per_rank;
-        const int rem = i - r * per_rank;
-        const int s = rem / P.Er;
-        const int e = r * P.Er + (rem - s * P.Er);
-        int cnt = 0;
-        for (int p = 0; p < P.P; ++p) cnt += __ldcg(P.partc + (size_t)(s * P.P + p) * P.E + e);
-        P.src_counts[(size_t)s * P.E + e] = cnt;
-        const int64_t rows = C > 0 ? C : (int64_t)((cnt + P.align - 1) / P.align) * P.align;
-        const int64_t kept = (C > 0 && cnt > C) ? C : cnt;
-        v[u] = (rows << 32) | kept;
-      }
-      local += v[u];
+  for (int u = 0; u < kChunkSeg / kSrcThreads; ++u) {
+    const int i = c0 + u * kSrcThreads + threadIdx.x;
+    if (i < nseg) {
+      int s, e;
+      seg_coords(P, i, s, e);
+      int cnt = 0;
+      for (int p = 0; p < P.P; ++p) cnt += __ldcg(P.partc + (size_t)(s * P.P + p) * P.E + e);
+      P.cnt[i] = cnt;
+      P.src_counts[(size_t)s * P.E + e] = cnt;
+      local += seg_value(P, cnt);
     }
-    int64_t total;
-    const int64_t incl = scan_block64(local, wsum, &total);
-    int64_t run = carry + incl - local;
+  }
+  const int64_t tot = sum_block64(local, wsum);
+  if (threadIdx.x == 0) P.blocksum[blockIdx.x] = tot;
+}
+
+// One CTA per chunk: the sums of the earlier chunks, then an exclusive scan
+// of the chunk's segments (kSegPerThread consecutive ones per thread) into
+// seg_off and the kept-row prefix.
+__global__ void __launch_bounds__(kSrcThreads) src_scan_kernel(const SrcParams P) {
+  __shared__ int64_t wsum[kSrcWarps];
+  pdl_wait();  // the totals are complete
+  pdl_trigger();
+  const int nseg = P.R * P.E;
+  int64_t pre = 0;
+  for (int c = threadIdx.x; c < (int)blockIdx.x; c += kSrcThreads) pre += __ldcg(P.blocksum + c);
+  pre = sum_block64(pre, wsum);
+  const int i0 = blockIdx.x * kChunkSeg + threadIdx.x * kSegPerThread;
+  int64_t v[kSegPerThread];
+  int64_t local = 0;
 #pragma unroll
-    for (int u = 0; u < kScanPer; ++u) {
-      const int i = c0 + threadIdx.x * kScanPer + u;
-      if (i < nseg) {
-        P.seg_off[i] = (int32_t)(run >> 32);
-        P.keptcum[i] = (int32_t)(run & 0xffffffffll);
-      }
-      run += v[u];
+  for (int u = 0; u < kSegPerThread; ++u) {
+    v[u] = (i0 + u < nseg) ? seg_value(P, __ldcg(P.cnt + i0 + u)) : 0;
+    local += v[u];
+  }
+  int64_t total;
+  int64_t run = pre + excl_scan_block64(local, wsum, &total);
+#pragma unroll
+  for (int u = 0; u < kSegPerThread; ++u) {
+    if (i0 + u < nseg) {
+      P.seg_off[i0 + u] = (int32_t)(run >> 32);
+      P.keptcum[i0 + u] = (int32_t)(run & 0xffffffffll);
     }
-    carry += total;
+    run += v[u];
   }
-  if (threadIdx.x == 0) {
-    P.seg_off[nseg] = (int32_t)(carry >> 32);
-    P.keptcum[nseg] = (int32_t)(carry & 0xffffffffll);
-  }
-  __syncthreads();  // this CTA's global writes above are visible below
-  for (int q = threadIdx.x; q < P.R * P.R; q += kScanThreads) {  // q = s*R + r
-    const int s = q / P.R, r = q - (q / P.R) * P.R;
-    const int lo = (r * P.R + s) * P.Er;
-    P.pair_counts[q] = __ldcg(P.keptcum + lo + P.Er) - __ldcg(P.keptcum + lo);
-  }
-  for (int r = threadIdx.x; r <= P.R; r += kScanThreads) {
-    P.rank_off[r] = __ldcg(P.seg_off + (size_t)r * per_rank);
-    if (r < P.R)
-      P.rank_counts[r] =
-          __ldcg(P.keptcum + (size_t)(r + 1) * per_rank) - __ldcg(P.keptcum + (size_t)r * per_rank);
+  if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) {
+    P.seg_off[nseg] = (int32_t)((pre + total) >> 32);
+    P.keptcum[nseg] = (int32_t)((pre + total) & 0xffffffffll);
   }
 }
 
@@ -189,6 +223,23 @@ __global__ void __launch_bounds__(kSrcThreads) src_place_kernel(const SrcParams 
   const int64_t i0 = (int64_t)t0 * P.k, i1 = (int64_t)t1 * P.k;
   pdl_wait();  // the scan (and, before it, the part counts) are complete
   pdl_trigger();
+  // message sizes and rank slices from the kept-row prefix (grid-stride)
+  {
+    const int per_rank = P.R * P.Er;
+    const int nthr = gridDim.x * kSrcThreads;
+    const int tid = b * kSrcThreads + threadIdx.x;
+    for (int q = tid; q < P.R * P.R; q += nthr) {  // q = s*R + r
+      const int sq = q / P.R, r = q - (q / P.R) * P.R;
+      const int lo = (r * P.R + sq) * P.Er;
+      P.pair_counts[q] = __ldcg(P.keptcum + lo + P.Er) - __ldcg(P.keptcum + lo);
+    }
+    for (int r = tid; r <= P.R; r += nthr) {
+      P.rank_off[r] = __ldcg(P.seg_off + (size_t)r * per_rank);
+      if (r < P.R)
+        P.rank_counts[r] = __ldcg(P.keptcum + (size_t)(r + 1) * per_rank) -
+                           __ldcg(P.keptcum + (size_t)r * per_rank);
+    }
+  }
   for (int x = threadIdx.x; x < kSrcWarps * P.E; x += kSrcThreads) wc[x] = 0;
   for (int e = threadIdx.x; e < P.E; e += kSrcThreads) {
     int pre = 0;
@@ -205,20 +256,30 @@ __global__ void __launch_bounds__(kSrcThreads) src_place_kernel(const SrcParams 
   // rank of every assignment inside the warp's run; `emit` sees (i, e, rank)
   // with rank -1 for an invalid id
   auto run = [&](auto&& emit) {
-    for (int64_t r0 = s0; r0 < s1; r0 += 32) {
-      const int64_t i = r0 + lane;
-      const int e = i < s1 ? __ldg(P.ids + i) : -1;
-      const bool ok = i < s1 && (unsigned)e < (unsigned)P.E;
-      const unsigned active = __ballot_sync(kFull, ok);
-      int v = -1;
-      if (ok) {
-        const unsigned peers = __match_any_sync(active, e);
-        v = my[e] + __popc(peers & lanemask_lt());
-        __syncwarp(active);
-        if (lane == __ffs(peers) - 1) my[e] = v + __popc(peers);
+    for (int64_t r0 = s0; r0 < s1; r0 += 32 * kRounds) {
+      int ev[kRounds];
+#pragma unroll
+      for (int u = 0; u < kRounds; ++u) {  // loads of kRounds rounds in flight
+        const int64_t i = r0 + 32 * u + lane;
+        ev[u] = i < s1 ? __ldg(P.ids + i) : -1;
       }
-      __syncwarp();
-      if (i < s1) emit(i, e, v);
+#pragma unroll
+      for (int u = 0; u < kRounds; ++u) {
+        const int64_t i = r0 + 32 * u + lane;
+        if (r0 + 32 * u >= s1) break;  // warp-uniform
+        const int e = ev[u];
+        const bool ok = i < s1 && (unsigned)e < (unsigned)P.E;
+        const unsigned active = __ballot_sync(kFull, ok);
+        int v = -1;
+        if (ok) {
+          const unsigned peers = __match_any_sync(active, e);
+          v = my[e] + __popc(peers & lanemask_lt());
+          __syncwarp(active);
+          if (lane == __ffs(peers) - 1) my[e] = v + __popc(peers);
+        }
+        __syncwarp();
+        if (i < s1) emit(i, e, v);
+      }
     }
   };
   run([](int64_t, int, int) {});
@@ -281,7 +342,7 @@ __global__ void __launch_bounds__(kSrcThreads) src_place_kernel(const SrcParams 
 
 cudaError_t launch_layout_src(const LaunchEnv& env, const int32_t* ids, int T, int E, int k, int R,
                               int capacity, int align, int64_t N, int32_t* partc,
-                              int32_t* keptcum, WsHeader* hdr, int32_t* src_counts,
+                              int32_t* scratch, WsHeader* hdr, int32_t* src_counts,
                               int32_t* seg_off, int32_t* pair_counts, int32_t* rank_off,
                               int32_t* rank_counts, int32_t* dst_pos, int32_t* src_idx) {
   const SrcGeom g = layout_src_geom(T, R);
@@ -299,7 +360,9 @@ cudaError_t launch_layout_src(const LaunchEnv& env, const int32_t* ids, int T, i
   P.P = g.P;
   P.N = N;
   P.partc = partc;
-  P.keptcum = keptcum;
+  P.cnt = scratch;
+  P.keptcum = scratch + ((size_t)R * E + 3) / 4 * 4;
+  P.blocksum = reinterpret_cast<int64_t*>(P.keptcum + ((size_t)R * E + 1 + 3) / 4 * 4);
   P.hdr = hdr;
   P.src_counts = src_counts;
   P.seg_off = seg_off;
@@ -320,7 +383,10 @@ cudaError_t launch_layout_src(const LaunchEnv& env, const int32_t* ids, int T, i
   if (err != cudaSuccess) return err;
   err = launch_pdl(env, src_count_kernel, dim3(parts), dim3(kSrcThreads), count_smem, P);
   if (err != cudaSuccess) return err;
-  err = launch_pdl(env, src_scan_kernel, dim3(1), dim3(kScanThreads), 0, P);
+  const unsigned chunks = (unsigned)(((int64_t)R * E + kChunkSeg - 1) / kChunkSeg);
+  err = launch_pdl(env, src_reduce_kernel, dim3(chunks), dim3(kSrcThreads), 0, P);
+  if (err != cudaSuccess) return err;
+  err = launch_pdl(env, src_scan_kernel, dim3(chunks), dim3(kSrcThreads), 0, P);
   if (err != cudaSuccess) return err;
   return launch_pdl(env, src_place_kernel, dim3(parts), dim3(kSrcThreads), place_smem, P);
 }

@@ -67,6 +67,23 @@ class Workload:
             return self.E * self.capacity
         return self.T * self.k + self.E * (self.align - 1)
 
+    @property
+    def capacity_src(self) -> int:
+        """Per-(source shard, expert) slots for the per-source-rank layout:
+        C = ceil(cf * Ts * k / E) with Ts = ceil(T/R) tokens per shard; 0 means
+        dropless."""
+        if self.capacity_factor is None:
+            return 0
+        ts = -(-self.T // self.R) if self.T > 0 else 1
+        return max(1, math.ceil(Fraction(self.capacity_factor) * ts * self.k / self.E))
+
+    @property
+    def rows_src(self) -> int:
+        """Rows of the per-source-rank layout (segments per (rank, shard, expert))."""
+        if self.capacity_src:
+            return self.R * self.E * self.capacity_src
+        return self.T * self.k + self.R * self.E * (self.align - 1)
+
     def with_(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
 

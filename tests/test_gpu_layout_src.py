@@ -84,7 +84,7 @@ def test_layout_src_full_size_on_routed_ids(wname):
     w = WORKLOADS[wname]
     inp = make_inputs(w)
     dev = torch.device("cuda:0")
-    shape = _shape(w.T, w.H, w.E, w.k, w.R, w.capacity, w.align, w.fp8)
+    shape = _shape(w.T, w.H, w.E, w.k, w.R, w.capacity_src, w.align, w.fp8)
     ws = m.Workspace(shape, dev)
     ids, _ = m.moe_route(shape, inp.logits.to(dev),
                          inp.bias.to(dev) if inp.bias is not None else None, ws=ws)
@@ -93,7 +93,8 @@ def test_layout_src_full_size_on_routed_ids(wname):
     lay = m.moe_layout_src(shape, ids, ws=ws)
     torch.cuda.synchronize()
     assert m.moe_get_device_error(ws) == (0, 0)
-    _compare(lay, oracle.layout_src(ids_np, w.E, w.R, capacity=w.capacity, align=w.align), wname)
+    _compare(lay, oracle.layout_src(ids_np, w.E, w.R, capacity=w.capacity_src, align=w.align),
+             wname)
 
 
 def test_empty_batch():
@@ -142,7 +143,7 @@ def test_dispatch_and_combine_over_the_src_layout(capacity_factor):
                  shared=True, residual=True, expert="scale")
     inp = make_inputs(w)
     dev = torch.device("cuda:0")
-    C = 0 if capacity_factor is None else int(np.ceil(capacity_factor * (w.T // w.R) * w.k / w.E))
+    C = w.capacity_src
     shape = _shape(w.T, w.H, w.E, w.k, w.R, C)
     ws = m.Workspace(shape, dev)
     x = inp.x.to(dev)
