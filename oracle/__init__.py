@@ -30,6 +30,8 @@ def lib():
         vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
         L.orc_route.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp]
         L.orc_route.restype = i32
+        L.orc_route_limited.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]
+        L.orc_route_limited.restype = i32
         L.orc_layout_rows.argtypes = [i32, i32, i32, i32, i32]
         L.orc_layout_rows.restype = i64
         L.orc_layout.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
@@ -81,6 +83,21 @@ def route(logits, k, bias=None, renorm=True):
     rc = lib().orc_route(T, E, k, int(bool(renorm)), _p(logits), _p(bias), _p(ids), _p(gates))
     if rc:
         raise OracleError(f"orc_route status {rc}")
+    return ids, gates
+
+
+def route_limited(logits, k, R, M, bias=None, renorm=True):
+    """Rank-limited route: experts from at most M of the R ranks (group score
+    = largest key on the rank).  Returns (ids int32 [T,k], gates fp32 [T,k])."""
+    logits = _c(logits, np.float32)
+    T, E = logits.shape
+    b = None if bias is None else _c(bias, np.float32)
+    ids = np.empty((T, k), np.int32)
+    gates = np.empty((T, k), np.float32)
+    rc = lib().orc_route_limited(T, E, k, R, M, 1 if renorm else 0, _p(logits), _p(b), _p(ids),
+                                 _p(gates))
+    if rc:
+        raise OracleError(f"orc_route_limited status {rc}")
     return ids, gates
 
 

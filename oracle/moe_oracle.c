@@ -37,6 +37,13 @@
  *   [MSG]  "GPU MoE all-to-all", section "The message-size distribution is
  *          the whole story": an all-to-all over a group of ranks is one
  *          logical message per (sender, receiver) pair, whatever the batch.
+ *   [NODE] "19. All-to-all", opening section: each token is limited to at
+ *          most 4 nodes so the slow hop stays bounded; section "Why Qwen3.8's
+ *          512 experts is a systems statement": node-limited routing as an
+ *          architectural constraint; "GPU MoE all-to-all", section "The node
+ *          boundary is the design decision": a token whose top-k experts sit
+ *          inside one node never crosses the NIC.  The pages give no group
+ *          score; the one used here is the largest key on the rank.
  *   [OCP]  OCP 8-bit Floating Point Specification (OFP8), E4M3 format:
  *          exponent bias 7, 3 mantissa bits, no infinities, S.1111.111 is
  *          NaN, largest finite magnitude 448, smallest subnormal 2^-9.
@@ -206,6 +213,89 @@ int orc_route(int T, int E, int k, int renorm, const float* logits, const float*
   }
   free(key);
   free(taken);
+  return ORC_OK;
+}
+
+/* Rank-limited route.  [NODE], [BIAS]
+ * As orc_route, except that each token's experts come from at most M of the
+ * R ranks (expert e lives on rank e / (E/R)):
+ *   score_r = max over the experts e of rank r of key_e;
+ *   the M ranks with the largest scores are eligible (equal scores: the
+ *   lower rank id first);
+ *   slots  = the k largest keys among the eligible ranks' experts (equal
+ *            keys: the lower expert id first);
+ *   gates  = as orc_route (raw logits; renorm over the k selected, else the
+ *            softmax over all E read at the selected ones).
+ * Needs 1 <= M, and k <= M * (E/R) so that k experts are eligible.  M >= R
+ * is the unrestricted route. */
+int orc_route_limited(int T, int E, int k, int R, int M, int renorm, const float* logits,
+                      const float* bias, int32_t* ids, float* gates) {
+  if (T < 0 || E < 1 || k < 1 || k > E || R < 1 || E % R != 0 || M < 1) return ORC_BAD_ARG;
+  const int Er = E / R;
+  if (M < R && k > M * Er) return ORC_BAD_ARG;
+  float* key = (float*)malloc(sizeof(float) * (size_t)E);
+  unsigned char* taken = (unsigned char*)malloc((size_t)E);
+  float* score = (float*)malloc(sizeof(float) * (size_t)R);
+  unsigned char* chosen = (unsigned char*)malloc((size_t)R);
+  if (!key || !taken || !score || !chosen) {
+    free(key); free(taken); free(score); free(chosen);
+    return ORC_BAD_ARG;
+  }
+  for (int t = 0; t < T; ++t) {
+    const float* lg = logits + (size_t)t * E;
+    for (int e = 0; e < E; ++e) {
+      key[e] = lg[e] + (bias ? bias[e] : 0.0f);
+      taken[e] = 0;
+    }
+    if (M < R) {
+      /* group score per rank, then the M best ranks */
+      for (int r = 0; r < R; ++r) {
+        score[r] = key[r * Er];
+        for (int e = r * Er + 1; e < (r + 1) * Er; ++e)
+          if (key[e] > score[r]) score[r] = key[e];
+        chosen[r] = 0;
+      }
+      for (int m = 0; m < M; ++m) {
+        int best = -1;
+        for (int r = 0; r < R; ++r) {
+          if (chosen[r]) continue;
+          if (best < 0 || score[r] > score[best]) best = r; /* strict: lower id on ties */
+        }
+        chosen[best] = 1;
+      }
+      /* experts of the other ranks cannot be selected */
+      for (int e = 0; e < E; ++e)
+        if (!chosen[e / Er]) taken[e] = 1;
+    }
+    for (int j = 0; j < k; ++j) {
+      int best = -1;
+      for (int e = 0; e < E; ++e) {
+        if (taken[e]) continue;
+        if (best < 0 || key[e] > key[best]) best = e;
+      }
+      taken[best] = 1;
+      ids[(size_t)t * k + j] = best;
+    }
+    double m = -INFINITY;
+    if (renorm) {
+      for (int j = 0; j < k; ++j) {
+        double l = (double)lg[ids[(size_t)t * k + j]];
+        if (l > m) m = l;
+      }
+      double den = 0.0;
+      for (int j = 0; j < k; ++j) den += exp((double)lg[ids[(size_t)t * k + j]] - m);
+      for (int j = 0; j < k; ++j)
+        gates[(size_t)t * k + j] = (float)(exp((double)lg[ids[(size_t)t * k + j]] - m) / den);
+    } else {
+      for (int e = 0; e < E; ++e)
+        if ((double)lg[e] > m) m = (double)lg[e];
+      double den = 0.0;
+      for (int e = 0; e < E; ++e) den += exp((double)lg[e] - m);
+      for (int j = 0; j < k; ++j)
+        gates[(size_t)t * k + j] = (float)(exp((double)lg[ids[(size_t)t * k + j]] - m) / den);
+    }
+  }
+  free(key); free(taken); free(score); free(chosen);
   return ORC_OK;
 }
 
