@@ -27,7 +27,7 @@ from . import _binding
 from ._binding import MoeError, MOE_F_FP8, MOE_F_RENORM, MOE_F_SRC_LAYOUT
 
 __all__ = ["MoeShape", "Workspace", "Layout", "LayoutSrc", "MoeError", "moe_route", "moe_layout",
-           "moe_layout_src",
+           "moe_layout_src", "moe_route_limited",
            "moe_route_layout", "moe_route_layout_dispatch",
            "moe_dispatch", "moe_combine", "moe_get_device_error", "moe_check",
            "moe_layout_rows", "moe_workspace_bytes"]
@@ -138,6 +138,25 @@ def moe_route(shape: MoeShape, logits: torch.Tensor, bias: Optional[torch.Tensor
         _ptr(bias, "bias", torch.float32, (E,)), _ptr(ids, "ids", torch.int32, (T, k)),
         _ptr(gates, "gates", torch.float32, (T, k)), ws.ptr, ws.nbytes, _stream(dev))
     _check(st, "moe_route")
+    return ids, gates
+
+
+def moe_route_limited(shape: MoeShape, logits: torch.Tensor, max_ranks: int,
+                      bias: Optional[torch.Tensor] = None, *, ws: Workspace,
+                      ids: Optional[torch.Tensor] = None, gates: Optional[torch.Tensor] = None):
+    """moe_route with each token's experts taken from at most `max_ranks` ranks."""
+    T, E, k = shape.tokens, shape.experts, shape.k
+    dev = logits.device
+    if ids is None:
+        ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    if gates is None:
+        gates = torch.empty((T, k), dtype=torch.float32, device=dev)
+    st = _binding.lib().moe_route_limited(
+        ctypes.byref(shape.c()), _ptr(logits, "logits", torch.float32, (T, E)),
+        _ptr(bias, "bias", torch.float32, (E,)), int(max_ranks),
+        _ptr(ids, "ids", torch.int32, (T, k)), _ptr(gates, "gates", torch.float32, (T, k)),
+        ws.ptr, ws.nbytes, _stream(dev))
+    _check(st, "moe_route_limited")
     return ids, gates
 
 

@@ -135,6 +135,26 @@ moe_status_t moe_route(const moe_shape_t* shape, const float* logits, const floa
                                      static_cast<WsHeader*>(ws)));
 }
 
+moe_status_t moe_route_limited(const moe_shape_t* shape, const float* logits, const float* bias,
+                               int32_t max_ranks, int32_t* ids, float* gates, void* ws,
+                               size_t ws_bytes, moe_stream_t stream) {
+  if (!shape_ok(shape) || max_ranks < 1) return MOE_ERR_INVALID_ARG;
+  const int R = shape->ranks, Er = shape->experts / shape->ranks;
+  if (max_ranks < R && shape->k > (int64_t)max_ranks * Er) return MOE_ERR_INVALID_ARG;
+  if (shape->tokens > 0 && (logits == nullptr || ids == nullptr || gates == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(logits, 4) || !aligned(bias, 4) || !aligned(ids, 4) || !aligned(gates, 4))
+    return MOE_ERR_INVALID_ARG;
+  moe_status_t st = ws_ok(shape, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  if (shape->tokens == 0) return MOE_OK;
+  return from_cuda(moe::launch_route(env_of(stream), logits, bias, shape->tokens,
+                                     shape->experts, shape->k,
+                                     (shape->flags & MOE_F_RENORM) ? 1 : 0, ids, gates,
+                                     static_cast<WsHeader*>(ws), nullptr, 0, R,
+                                     max_ranks < R ? max_ranks : 0));
+}
+
 moe_status_t moe_layout(const moe_shape_t* shape, const int32_t* ids, int32_t* counts,
                         int32_t* expert_off, int32_t* rank_off, int32_t* rank_counts,
                         int32_t* dst_pos, int32_t* src_idx, void* ws, size_t ws_bytes,

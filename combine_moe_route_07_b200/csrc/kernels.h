@@ -112,10 +112,12 @@ cudaError_t launch_layout_src(const LaunchEnv& env, const int32_t* ids, int T, i
 
 // tables != nullptr: also add each routed token's ids into the layout tile
 // table the next place pass reads (the fused route + layout path).  `tables`
-// holds two tables of `half_words` words each.
+// holds two tables of `half_words` words each.  0 < max_ranks < R: each
+// token's experts come from at most max_ranks of the R ranks.
 cudaError_t launch_route(const LaunchEnv& env, const float* logits, const float* bias, int T,
                          int E, int k, int renorm, int32_t* ids, float* gates, WsHeader* hdr,
-                         uint32_t* tables = nullptr, size_t half_words = 0);
+                         uint32_t* tables = nullptr, size_t half_words = 0, int R = 1,
+                         int max_ranks = 0);
 
 // Layout of `ids` (count pass + place pass).  count_ids == false: the tile
 // table was already filled by a route launch with tables (fused path).

@@ -32,8 +32,9 @@ __global__ void __launch_bounds__(kThreads)
     route_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E,
                  int k, int renorm, int32_t* __restrict__ ids, float* __restrict__ gates,
                  WsHeader* hdr, uint32_t* __restrict__ tables, int TT, size_t table_words,
-                 int per) {
-  // dynamic: [hist: E int32, padded to 16 B] (HIST), [rows: kWarps x 2 x E floats] (STAGE)
+                 int per, int R, int M) {
+  // dynamic: [hist: E int32, padded to 16 B] (HIST), [rows: kWarps x 2 x E floats] (STAGE),
+  // [rank limit: kWarps x (R + ceil(R/32)) words] (M < R)
   extern __shared__ __align__(16) unsigned char dyn[];
   __shared__ uint32_t cand_all[kWarps][NK >= 8 ? 3 * kMaxCand : 1];
   __shared__ uint64_t bars[kWarps][2];
@@ -41,6 +42,15 @@ __global__ void __launch_bounds__(kThreads)
   const size_t hist_bytes = HIST ? (((size_t)E * 4 + 15) & ~(size_t)15) : 0;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   float* buf = reinterpret_cast<float*>(dyn + hist_bytes) + (size_t)w * 2 * E;
+  RankLimit lim;
+  lim.R = R;
+  lim.M = M;
+  if (lim.on()) {
+    const size_t lim_words = (size_t)R + (R + 31) / 32;
+    lim.smem = reinterpret_cast<uint32_t*>(dyn + hist_bytes +
+                                           (STAGE ? (size_t)kWarps * 2 * E * sizeof(float) : 0)) +
+               (size_t)w * lim_words;
+  }
   if (STAGE && lane == 0) {
     mbar_init(&bars[w][0], 1);
     mbar_init(&bars[w][1], 1);
@@ -111,17 +121,18 @@ __global__ void __launch_bounds__(kThreads)
           parity ^= 1u << sb;
           pending &= ~(1u << sb);
           nan_tok = route_token_thr<NK, true>(logits, t, T, b, E, k, renorm, lane, cand_all[w],
-                                              e1, g1, buf + (size_t)sb * E);
+                                              e1, g1, buf + (size_t)sb * E, lim);
         } else {
           if (lane == 0) report(hdr, MOE_ERR_DEVICE_TIMEOUT, t);
           alive = false;  // routes nothing more; still takes part in the CTA barriers
         }
       } else if constexpr (NK >= 8) {
-        nan_tok = route_token_thr<NK>(logits, t, T, b, E, k, renorm, lane, cand_all[w], e1, g1);
+        nan_tok = route_token_thr<NK>(logits, t, T, b, E, k, renorm, lane, cand_all[w], e1, g1,
+                                      nullptr, lim);
       } else {
         int tok[1] = {t}, ea[1];
         float ga[1];
-        nan_tok = route_tokens<NK, 1>(logits, tok, T, b, E, k, renorm, lane, ea, ga);
+        nan_tok = route_tokens<NK, 1>(logits, tok, T, b, E, k, renorm, lane, ea, ga, lim);
         e1 = ea[0];
         g1 = ga[0];
       }
@@ -150,12 +161,14 @@ __global__ void __launch_bounds__(kThreads)
 template <int NK, bool HIST>
 cudaError_t launch_nk(const LaunchEnv& env, const float* logits, const float* bias, int T, int E,
                       int k, int renorm, int32_t* ids, float* gates, WsHeader* hdr,
-                      uint32_t* tables, int TT, size_t table_words) {
+                      uint32_t* tables, int TT, size_t table_words, int R, int M) {
   const size_t hist_bytes = HIST ? (((size_t)E * 4 + 15) & ~(size_t)15) : 0;
   // rows staged by bulk copy: many keys per lane, 16-byte rows and base
   const bool stage = NK >= 8 && (E % 4) == 0 && (reinterpret_cast<uintptr_t>(logits) & 15u) == 0;
   auto kern = stage ? route_kernel<NK, HIST, NK >= 8> : route_kernel<NK, HIST, false>;
-  const size_t smem = hist_bytes + (stage ? (size_t)kWarps * 2 * E * sizeof(float) : 0);
+  const bool limit = M > 0 && M < R;
+  const size_t smem = hist_bytes + (stage ? (size_t)kWarps * 2 * E * sizeof(float) : 0) +
+                      (limit ? (size_t)kWarps * (R + (R + 31) / 32) * sizeof(uint32_t) : 0);
   int per_sm = 1;
   const cudaError_t err = blocks_per_sm(reinterpret_cast<const void*>(kern), kThreads, smem, &per_sm);
   if (err != cudaSuccess) return err;
@@ -170,18 +183,18 @@ cudaError_t launch_nk(const LaunchEnv& env, const float* logits, const float* bi
   blocks = ((int64_t)T + per - 1) / per;
   if (blocks < 1) blocks = 1;
   return launch_pdl(env, kern, dim3((unsigned)blocks), dim3(kThreads), smem, logits, bias, T, E,
-                    k, renorm, ids, gates, hdr, tables, TT, table_words, (int)per);
+                    k, renorm, ids, gates, hdr, tables, TT, table_words, (int)per, R, M);
 }
 
 template <bool HIST>
 cudaError_t launch_any(const LaunchEnv& env, const float* logits, const float* bias, int T, int E,
                        int k, int renorm, int32_t* ids, float* gates, WsHeader* hdr,
-                       uint32_t* tables, int TT, size_t table_words) {
+                       uint32_t* tables, int TT, size_t table_words, int R, int M) {
   const int nk = (E + 31) / 32;
 #define MOE_ROUTE_NK(N)                                                                         \
   if (nk <= N)                                                                                  \
     return launch_nk<N, HIST>(env, logits, bias, T, E, k, renorm, ids, gates, hdr, tables, TT, \
-                              table_words);
+                              table_words, R, M);
   MOE_ROUTE_NK(1)
   MOE_ROUTE_NK(2)
   MOE_ROUTE_NK(4)
@@ -189,19 +202,20 @@ cudaError_t launch_any(const LaunchEnv& env, const float* logits, const float* b
   MOE_ROUTE_NK(16)
 #undef MOE_ROUTE_NK
   return launch_nk<32, HIST>(env, logits, bias, T, E, k, renorm, ids, gates, hdr, tables, TT,
-                             table_words);
+                             table_words, R, M);
 }
 
 }  // namespace
 
 cudaError_t launch_route(const LaunchEnv& env, const float* logits, const float* bias, int T,
                          int E, int k, int renorm, int32_t* ids, float* gates, WsHeader* hdr,
-                         uint32_t* tables, size_t half_words) {
+                         uint32_t* tables, size_t half_words, int R, int max_ranks) {
   if (tables == nullptr)
-    return launch_any<false>(env, logits, bias, T, E, k, renorm, ids, gates, hdr, nullptr, 1, 0);
+    return launch_any<false>(env, logits, bias, T, E, k, renorm, ids, gates, hdr, nullptr, 1, 0,
+                             R, max_ranks);
   const TileGeom geom = layout_tiles(T);
   return launch_any<true>(env, logits, bias, T, E, k, renorm, ids, gates, hdr, tables, geom.TT,
-                          half_words);
+                          half_words, R, max_ranks);
 }
 
 }  // namespace moe

@@ -49,6 +49,63 @@ __device__ __forceinline__ void load_bias(const float* bias, int E, int lane, fl
   }
 }
 
+// Rank limit: each token's experts come from at most M of the R ranks (expert
+// e on rank e / (E/R)).  Group score of a rank = its largest key code; the M
+// best ranks are kept (equal scores: the lower rank id), every other rank's
+// codes are cleared to 0 ("taken") before the selection.  "19. All-to-all",
+// opening section (each token limited to a few nodes); "GPU MoE all-to-all",
+// section "The node boundary is the design decision".  `smem` is this warp's
+// R + ceil(R/32) words.  Off when M <= 0 or M >= R.
+struct RankLimit {
+  int R = 1;
+  int M = 0;
+  uint32_t* smem = nullptr;
+  __device__ bool on() const { return M > 0 && M < R; }
+};
+
+template <int NK>
+__device__ __forceinline__ void apply_rank_limit(uint32_t (&code)[NK], int E, int lane,
+                                                 const RankLimit& L) {
+  const int R = L.R, Er = E / R;
+  uint32_t* rmax = L.smem;
+  uint32_t* chosen = L.smem + R;  // bitmap of the kept ranks
+  for (int r = lane; r < R; r += 32) rmax[r] = 0u;
+  for (int q = lane; q < (R + 31) / 32; q += 32) chosen[q] = 0u;
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < NK; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E && code[i] != 0u) atomicMax(&rmax[e / Er], code[i]);
+  }
+  __syncwarp();
+  for (int m = 0; m < L.M; ++m) {
+    uint32_t best = 0u;
+    int bi = R;
+    for (int r = lane; r < R; r += 32) {  // ascending r: strict > keeps the lower id
+      if (((chosen[r >> 5] >> (r & 31)) & 1u) == 0u) {
+        const uint32_t v = rmax[r];
+        if (bi == R || v > best) {
+          best = v;
+          bi = r;
+        }
+      }
+    }
+    const uint32_t top = __reduce_max_sync(kFull, best);
+    const uint32_t win = __reduce_min_sync(kFull, (bi < R && best == top) ? (uint32_t)bi : 0xffffffffu);
+    if (lane == 0) chosen[win >> 5] |= 1u << (win & 31u);
+    __syncwarp();
+  }
+#pragma unroll
+  for (int i = 0; i < NK; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E) {
+      const int r = e / Er;
+      if (((chosen[r >> 5] >> (r & 31)) & 1u) == 0u) code[i] = 0u;
+    }
+  }
+  __syncwarp();  // the next token reuses the words
+}
+
 // Tokens per warp group for NK keys per lane (register budget).
 template <int NK>
 struct RouteGroup {
@@ -61,7 +118,8 @@ struct RouteGroup {
 template <int NK, int TPW>
 __device__ __forceinline__ int route_tokens(const float* __restrict__ logits, const int (&tok)[TPW],
                                             int T, const float (&b)[NK], int E, int k, int renorm,
-                                            int lane, int (&sel_e)[TPW], float (&gate)[TPW]) {
+                                            int lane, int (&sel_e)[TPW], float (&gate)[TPW],
+                                            const RankLimit& lim = RankLimit()) {
   float raw[TPW][NK];
   uint32_t code[TPW][NK];
   int nan_tok = -1;
@@ -84,6 +142,7 @@ __device__ __forceinline__ int route_tokens(const float* __restrict__ logits, co
       }
     }
     if (__any_sync(kFull, bad) && nan_tok < 0) nan_tok = tok[u];
+    if (lim.on()) apply_rank_limit<NK>(code[u], E, lane, lim);
   }
 
   float sel_raw[TPW];
@@ -160,7 +219,8 @@ template <int NK, bool SMEM = false>
 __device__ __forceinline__ int route_token_thr(const float* __restrict__ logits, int t, int T,
                                                const float (&b)[NK], int E, int k, int renorm,
                                                int lane, uint32_t* cand, int& sel_e,
-                                               float& gate, const float* srow = nullptr) {
+                                               float& gate, const float* srow = nullptr,
+                                               const RankLimit& lim = RankLimit()) {
   float raw[NK];
   uint32_t code[NK];
   bool bad = false;
@@ -179,6 +239,7 @@ __device__ __forceinline__ int route_token_thr(const float* __restrict__ logits,
     }
   }
   const int nan_tok = __any_sync(kFull, bad) ? t : -1;
+  if (lim.on()) apply_rank_limit<NK>(code, E, lane, lim);
 
   // threshold: k-th largest lane maximum
   uint32_t mm = 0u;
@@ -198,7 +259,7 @@ __device__ __forceinline__ int route_token_thr(const float* __restrict__ logits,
   if (total > kMaxCand) {  // heavy ties at the threshold: the full scan
     int tok[1] = {t}, e1[1];
     float g1[1];
-    route_tokens<NK, 1>(logits, tok, T, b, E, k, renorm, lane, e1, g1);
+    route_tokens<NK, 1>(logits, tok, T, b, E, k, renorm, lane, e1, g1, lim);
     sel_e = e1[0];
     gate = g1[0];
     return nan_tok;

@@ -119,6 +119,24 @@ moe_status_t moe_route(const moe_shape_t* shape, const float* logits, const floa
                        int32_t* ids, float* gates, void* ws, size_t ws_bytes,
                        moe_stream_t stream);
 
+/* Step 1 with rank-limited (node-limited) routing: each token's k experts
+ * come from at most `max_ranks` of the R ranks ("19. All-to-all", opening
+ * section: tokens limited to at most a few nodes so the slow hop stays
+ * bounded; section "Why Qwen3.8's 512 experts is a systems statement":
+ * node-limited routing as a constraint; "GPU MoE all-to-all", section "The
+ * node boundary is the design decision").  The pages give no rank score; the
+ * one used here is the largest key on the rank:
+ *   score[r]  = max over the experts e of rank r of key[e]
+ *   the max_ranks ranks with the largest scores are eligible (equal scores:
+ *   the lower rank id); ids = the k largest keys among their experts (equal
+ *   keys: the lower expert id); gates as moe_route.
+ * 1 <= max_ranks; when max_ranks < R, k <= max_ranks * (E/R) is required
+ * (else MOE_ERR_INVALID_ARG).  max_ranks >= R is exactly moe_route.  Same
+ * buffers, layouts and errors as moe_route. */
+moe_status_t moe_route_limited(const moe_shape_t* shape, const float* logits, const float* bias,
+                               int32_t max_ranks, int32_t* ids, float* gates, void* ws,
+                               size_t ws_bytes, moe_stream_t stream);
+
 /* Steps 2 and 3 -- count histogram and layout scan ("GPU MoE all-to-all",
  * sections "Two collectives per layer" and "Bucketing"; "MoE All-to-All
  * Dispatch and Ragged Routing", section "Fixed Capacity vs. Ragged Routing").
