@@ -50,6 +50,9 @@ def parse():
                    help="expert: rows by expert; src: the per-source-rank layout (rows by "
                         "destination rank, source shard, expert), route + layout_src + dispatch "
                         "+ combine as separate calls")
+    p.add_argument("--max-ranks", type=int, default=0,
+                   help="> 0: rank-limited routing (moe_route_limited), each token's experts from "
+                        "at most this many ranks; route, layout, dispatch, combine as separate calls")
     p.add_argument("--tokens", type=int, default=0,
                    help="override the workload's token count (smaller cases for profiler "
                         "captures; a changed workload, not a bench line)")
@@ -69,6 +72,7 @@ def algorithmic_bytes(w, kept_rows):
     disp_row_out = (H + 4 * (H // 128)) if w.fp8 else row
     b = {}
     b["route"] = T * E * 4 + (4 * E if w.bias else 0) + T * k * 8
+    b["route_limited"] = b["route"]
     b["layout"] = T * k * 4 * 2 + w.rows * 4 + (3 * E + 2 * w.R) * 4  # ids in, dst_pos/src_idx out
     b["dispatch"] = T * row + kept_rows * disp_row_out + T * k * 4
     b["combine"] = kept_rows * row + T * k * 8 + T * row \
@@ -345,8 +349,16 @@ def main():
     shared = x if w.shared else None
     residual = x if w.residual else None
 
+    M = args.max_ranks
+
+    def route_op():
+        if M > 0:
+            m.moe_route_limited(shape, logits, M, bias, ws=ws, ids=ids, gates=gates)
+        else:
+            m.moe_route(shape, logits, bias, ws=ws, ids=ids, gates=gates)
+
     def route_layout_dispatch():
-        m.moe_route(shape, logits, bias, ws=ws, ids=ids, gates=gates)
+        route_op()
         if src:
             m.moe_layout_src(shape, ids, ws=ws, out=lay)
         else:
@@ -394,11 +406,13 @@ def main():
         lambda: m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared,
                               residual=residual, out=out),
     )
-    if src:
-        names = ("route", "layout_src", "dispatch", "combine")
+    if src or M > 0:
+        names = ("route_limited" if M > 0 else "route", "layout_src" if src else "layout",
+                 "dispatch", "combine")
         ops = (
-            lambda: m.moe_route(shape, logits, bias, ws=ws, ids=ids, gates=gates),
-            lambda: m.moe_layout_src(shape, ids, ws=ws, out=lay),
+            route_op,
+            (lambda: m.moe_layout_src(shape, ids, ws=ws, out=lay)) if src else
+            (lambda: m.moe_layout(shape, ids, ws=ws, out=lay)),
             lambda: m.moe_dispatch(shape, x, lay.dst_pos, ws=ws, out=xd, scales=sc),
             lambda: m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared,
                                   residual=residual, out=out),
@@ -480,8 +494,9 @@ def main():
     # per-kernel breakdown: a probe graph of the same step with event-record
     # nodes between the kernels, replayed after an L2 flush and read back one
     # replay at a time
-    probe_names = names if (src or args.path != "fused3") else names_probe
-    probe_ops = ops if (src or args.path != "fused3") else ops_probe
+    separate = src or M > 0
+    probe_names = names if (separate or args.path != "fused3") else names_probe
+    probe_ops = ops if (separate or args.path != "fused3") else ops_probe
     n_ops = len(probe_ops)
     probe_ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ops + 1)]
     g_probe = torch.cuda.CUDAGraph()
@@ -595,6 +610,7 @@ def main():
                    "layout": ("per-source-rank: rows by destination rank, source shard "
                               "(R shards of ceil(T/R) tokens), expert, token") if src else
                              "rows by expert, token",
+                   "max_ranks": M if M > 0 else None,
                    "step": " + ".join(names) + ", one CUDA graph"},
         "dispatch_combine": {"tokens_per_s": world * T / (dc_ms * 1e-3),
                              "us": round(dc_ms * 1e3, 2), "gbs": round(dc_gbs, 1),
@@ -622,7 +638,8 @@ def main():
                      "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
                      "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
                      "traffic": ncu_traffic(dom, w.name)},
-        "gpu_launches": (7 if src else {"fused3": 4, "fused": 4, "separate": 5}[args.path]) * K,
+        "gpu_launches": ((7 if src else 5) if separate else
+                         {"fused3": 4, "fused": 4, "separate": 5}[args.path]) * K,
         "clocks": clocks,
         "e2e": e2e,
     }

@@ -45,6 +45,7 @@ __global__ void __launch_bounds__(kThreads)
   RankLimit lim;
   lim.R = R;
   lim.M = M;
+  lim.init(E, lane);
   if (lim.on()) {
     const size_t lim_words = (size_t)R + (R + 31) / 32;
     lim.smem = reinterpret_cast<uint32_t*>(dyn + hist_bytes +

@@ -55,27 +55,120 @@ __device__ __forceinline__ void load_bias(const float* bias, int E, int lane, fl
 // codes are cleared to 0 ("taken") before the selection.  "19. All-to-all",
 // opening section (each token limited to a few nodes); "GPU MoE all-to-all",
 // section "The node boundary is the design decision".  `smem` is this warp's
-// R + ceil(R/32) words.  Off when M <= 0 or M >= R.
+// R + ceil(R/32) words (used only when E/R neither divides nor is a multiple
+// of 32).  Off when M <= 0 or M >= R.
 struct RankLimit {
   int R = 1;
   int M = 0;
   uint32_t* smem = nullptr;
+  // per-lane constants, set once by init(): experts per rank, how ranks map
+  // onto the lane-major keys, and this lane's place in that map
+  int Er = 1;
+  int mode = 0;  // 1: Er divides 32, R <= 64 (ranks inside a column); 2: whole columns; 0: other
+  int step = 0;  // mode 1: ranks per column; mode 2: columns per rank
+  int lane_rank = 0;
+  bool lead = false;
   __device__ bool on() const { return M > 0 && M < R; }
+  __device__ void init(int E, int lane) {
+    Er = E / R;
+    if (Er <= 32 && (32 % Er) == 0 && R <= 64) {
+      mode = 1;
+      step = 32 / Er;
+      lane_rank = lane / Er;
+      lead = (lane % Er) == 0;
+    } else if ((Er & 31) == 0) {
+      mode = 2;
+      step = Er >> 5;
+    } else {
+      mode = 0;
+    }
+  }
 };
 
 template <int NK>
 __device__ __forceinline__ void apply_rank_limit(uint32_t (&code)[NK], int E, int lane,
                                                  const RankLimit& L) {
-  const int R = L.R, Er = E / R;
+  const int R = L.R;
+  if (L.mode == 1) {
+    // A rank is Er aligned lanes of one column (R <= 64): an xor-max over the
+    // group gives the rank's score, the group's first lane stores it, and
+    // lane l then holds the scores of ranks l and l+32; M rounds of a warp
+    // arg-max (lower id on ties) fill a 64-bit mask of the kept ranks.
+    uint32_t* rmax = L.smem;
+#pragma unroll
+    for (int i = 0; i < NK; ++i) {
+      const bool valid = lane + 32 * i < E;
+      uint32_t v = valid ? code[i] : 0u;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1)
+        if (o < L.Er) v = max(v, __shfl_xor_sync(kFull, v, o));
+      if (valid && L.lead) rmax[i * L.step + L.lane_rank] = v;
+    }
+    __syncwarp();
+    const uint32_t s0 = lane < R ? rmax[lane] : 0u;
+    const uint32_t s1 = lane + 32 < R ? rmax[lane + 32] : 0u;
+    __syncwarp();  // the next token reuses the words
+    uint64_t kept = 0ull;
+    for (int m = 0; m < L.M; ++m) {
+      const uint32_t b0 = ((kept >> lane) & 1ull) ? 0u : s0;  // valid scores are never 0
+      const uint32_t b1 = ((kept >> (lane + 32)) & 1ull) ? 0u : s1;
+      const uint32_t best = max(b0, b1);
+      const uint32_t id = b0 >= b1 ? (uint32_t)lane : (uint32_t)(lane + 32);
+      const uint32_t top = __reduce_max_sync(kFull, best);
+      const uint32_t win = __reduce_min_sync(kFull, best == top ? id : 0xffffffffu);
+      kept |= 1ull << win;
+    }
+#pragma unroll
+    for (int i = 0; i < NK; ++i)
+      if (((kept >> (i * L.step + L.lane_rank)) & 1ull) == 0ull) code[i] = 0u;
+    return;
+  }
+  if (L.mode == 2) {
+    // A rank is Er/32 whole columns: every lane ends up with every score
+    // (R <= NK), so all lanes take the same M decisions without exchange.
+    uint32_t sc[NK];  // sc[i]: score of the rank whose last column is i
+    uint32_t acc = 0u;
+#pragma unroll
+    for (int i = 0; i < NK; ++i) {
+      sc[i] = 0u;
+      if (32 * i < E) {
+        acc = max(acc, code[i]);
+        if ((i + 1) % L.step == 0) {
+          sc[i] = __reduce_max_sync(kFull, acc);
+          acc = 0u;
+        }
+      }
+    }
+    uint32_t keep = 0u;  // bit i: the rank ending at column i is kept
+    for (int m = 0; m < L.M; ++m) {
+      uint32_t best = 0u;
+      int bi = -1;
+#pragma unroll
+      for (int i = 0; i < NK; ++i)
+        if (32 * i < E && (i + 1) % L.step == 0 && ((keep >> i) & 1u) == 0u &&
+            (bi < 0 || sc[i] > best)) {
+          best = sc[i];
+          bi = i;
+        }
+      keep |= 1u << bi;
+    }
+#pragma unroll
+    for (int i = 0; i < NK; ++i) {  // column i belongs to the rank ending at its group's last column
+      const int last = (i / L.step + 1) * L.step - 1;
+      if (last >= NK || ((keep >> last) & 1u) == 0u) code[i] = 0u;
+    }
+    return;
+  }
+  // other sizes: shared-memory maxima and a shared bitmap of kept ranks
   uint32_t* rmax = L.smem;
-  uint32_t* chosen = L.smem + R;  // bitmap of the kept ranks
-  for (int r = lane; r < R; r += 32) rmax[r] = 0u;
+  uint32_t* chosen = L.smem + R;
   for (int q = lane; q < (R + 31) / 32; q += 32) chosen[q] = 0u;
+  for (int r = lane; r < R; r += 32) rmax[r] = 0u;
   __syncwarp();
 #pragma unroll
   for (int i = 0; i < NK; ++i) {
     const int e = lane + 32 * i;
-    if (e < E && code[i] != 0u) atomicMax(&rmax[e / Er], code[i]);
+    if (e < E && code[i] != 0u) atomicMax(&rmax[e / L.Er], code[i]);
   }
   __syncwarp();
   for (int m = 0; m < L.M; ++m) {
@@ -91,7 +184,8 @@ __device__ __forceinline__ void apply_rank_limit(uint32_t (&code)[NK], int E, in
       }
     }
     const uint32_t top = __reduce_max_sync(kFull, best);
-    const uint32_t win = __reduce_min_sync(kFull, (bi < R && best == top) ? (uint32_t)bi : 0xffffffffu);
+    const uint32_t win =
+        __reduce_min_sync(kFull, (bi < R && best == top) ? (uint32_t)bi : 0xffffffffu);
     if (lane == 0) chosen[win >> 5] |= 1u << (win & 31u);
     __syncwarp();
   }
@@ -99,7 +193,7 @@ __device__ __forceinline__ void apply_rank_limit(uint32_t (&code)[NK], int E, in
   for (int i = 0; i < NK; ++i) {
     const int e = lane + 32 * i;
     if (e < E) {
-      const int r = e / Er;
+      const int r = e / L.Er;
       if (((chosen[r >> 5] >> (r & 31)) & 1u) == 0u) code[i] = 0u;
     }
   }
