@@ -32,6 +32,8 @@ def lib():
         L.orc_route.restype = i32
         L.orc_route_limited.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]
         L.orc_route_limited.restype = i32
+        L.orc_bias_update.argtypes = [i32, i64, vp, ctypes.c_float, vp, vp]
+        L.orc_bias_update.restype = None
         L.orc_layout_rows.argtypes = [i32, i32, i32, i32, i32]
         L.orc_layout_rows.restype = i64
         L.orc_layout.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
@@ -99,6 +101,17 @@ def route_limited(logits, k, R, M, bias=None, renorm=True):
     if rc:
         raise OracleError(f"orc_route_limited status {rc}")
     return ids, gates
+
+
+def bias_update(counts, assignments, gamma, bias):
+    """b_e + gamma * sign(assignments/E - counts[e]) (the aux-loss-free
+    balancing step); returns the new fp32 bias."""
+    counts = _c(counts, np.int32)
+    bias = _c(bias, np.float32)
+    E = counts.shape[0]
+    out = np.empty(E, np.float32)
+    lib().orc_bias_update(E, int(assignments), _p(counts), float(gamma), _p(bias), _p(out))
+    return out
 
 
 def layout_rows(T, E, k, capacity=0, align=1):

@@ -299,6 +299,28 @@ int orc_route_limited(int T, int E, int k, int R, int M, int renorm, const float
   return ORC_OK;
 }
 
+/* Aux-loss-free balancing: the per-expert bias update.  [BIAS]
+ * After a batch with load_e = counts[e] assignments per expert (before any
+ * drop) and mean = T*k/E, every bias moves by gamma towards balance:
+ *   b_e <- b_e + gamma * sign(mean - load_e)
+ * (an under-loaded expert's bias rises, an over-loaded one's falls, an
+ * expert exactly at the mean keeps its bias).  The sign is taken exactly, in
+ * integers: sign(T*k - E*load_e).  The update is one binary32 addition of
+ * +gamma, -gamma or nothing.  The pages give neither gamma nor the sign
+ * rule's form beyond "bump up or down based on recent load". */
+void orc_bias_update(int E, int64_t assignments, const int32_t* counts, float gamma,
+                     const float* bias_in, float* bias_out) {
+  for (int e = 0; e < E; ++e) {
+    const int64_t d = assignments - (int64_t)E * counts[e];
+    if (d > 0)
+      bias_out[e] = bias_in[e] + gamma;
+    else if (d < 0)
+      bias_out[e] = bias_in[e] - gamma;
+    else
+      bias_out[e] = bias_in[e];
+  }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Steps 2-3: count histogram and layout.  [TWO], [BUCK], [RAG], [OWN]       */
 /* ------------------------------------------------------------------------ */
