@@ -53,6 +53,10 @@ def parse():
     p.add_argument("--max-ranks", type=int, default=0,
                    help="> 0: rank-limited routing (moe_route_limited), each token's experts from "
                         "at most this many ranks; route, layout, dispatch, combine as separate calls")
+    p.add_argument("--bias-gamma", type=float, default=0.0,
+                   help="> 0: each step also runs the aux-loss-free bias update "
+                        "(moe_bias_update) with this step size; the bias feeds the next step's "
+                        "route")
     p.add_argument("--tokens", type=int, default=0,
                    help="override the workload's token count (smaller cases for profiler "
                         "captures; a changed workload, not a bench line)")
@@ -73,6 +77,7 @@ def algorithmic_bytes(w, kept_rows):
     b = {}
     b["route"] = T * E * 4 + (4 * E if w.bias else 0) + T * k * 8
     b["route_limited"] = b["route"]
+    b["bias_update"] = 12 * E  # counts in, bias in and out
     b["layout"] = T * k * 4 * 2 + w.rows * 4 + (3 * E + 2 * w.R) * 4  # ids in, dst_pos/src_idx out
     b["dispatch"] = T * row + kept_rows * disp_row_out + T * k * 4
     b["combine"] = kept_rows * row + T * k * 8 + T * row \
@@ -326,6 +331,9 @@ def main():
     x = inp.x.to(dev)
     logits = inp.logits.to(dev)
     bias = None if inp.bias is None else inp.bias.to(dev)
+    G = args.bias_gamma
+    if G > 0 and bias is None:
+        bias = torch.zeros(w.E, dtype=torch.float32, device=dev)
     T, k, N = w.T, w.k, shape.rows
     i32 = dict(dtype=torch.int32, device=dev)
     ids = torch.empty((T, k), **i32)
@@ -406,6 +414,10 @@ def main():
         lambda: m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared,
                               residual=residual, out=out),
     )
+    bias_op = lambda: m.moe_bias_update(shape, lay.counts, G, bias)  # noqa: E731
+    if G > 0:
+        names_probe = ("route_layout", "dispatch", "bias_update", "combine")
+        ops_probe = (ops_probe[0], ops_probe[1], bias_op, ops_probe[2])
     if src or M > 0:
         names = ("route_limited" if M > 0 else "route", "layout_src" if src else "layout",
                  "dispatch", "combine")
@@ -425,6 +437,9 @@ def main():
             lambda: m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared,
                                   residual=residual, out=out),
         )
+        if G > 0:
+            names = ("route_layout_dispatch", "bias_update", "combine")
+            ops = (ops[0], bias_op, ops[1])
     elif args.path == "fused":
         names = ("route_layout", "dispatch", "combine")
         ops = (
@@ -611,6 +626,7 @@ def main():
                               "(R shards of ceil(T/R) tokens), expert, token") if src else
                              "rows by expert, token",
                    "max_ranks": M if M > 0 else None,
+                   "bias_gamma": G if G > 0 else None,
                    "step": " + ".join(names) + ", one CUDA graph"},
         "dispatch_combine": {"tokens_per_s": world * T / (dc_ms * 1e-3),
                              "us": round(dc_ms * 1e3, 2), "gbs": round(dc_gbs, 1),
@@ -639,7 +655,8 @@ def main():
                      "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
                      "traffic": ncu_traffic(dom, w.name)},
         "gpu_launches": ((7 if src else 5) if separate else
-                         {"fused3": 4, "fused": 4, "separate": 5}[args.path]) * K,
+                         {"fused3": 4, "fused": 4, "separate": 5}[args.path] + (1 if G > 0 else 0))
+                        * K,
         "clocks": clocks,
         "e2e": e2e,
     }

@@ -27,7 +27,7 @@ from . import _binding
 from ._binding import MoeError, MOE_F_FP8, MOE_F_RENORM, MOE_F_SRC_LAYOUT
 
 __all__ = ["MoeShape", "Workspace", "Layout", "LayoutSrc", "MoeError", "moe_route", "moe_layout",
-           "moe_layout_src", "moe_route_limited",
+           "moe_layout_src", "moe_route_limited", "moe_bias_update",
            "moe_route_layout", "moe_route_layout_dispatch",
            "moe_dispatch", "moe_combine", "moe_get_device_error", "moe_check",
            "moe_layout_rows", "moe_workspace_bytes"]
@@ -158,6 +158,17 @@ def moe_route_limited(shape: MoeShape, logits: torch.Tensor, max_ranks: int,
         ws.ptr, ws.nbytes, _stream(dev))
     _check(st, "moe_route_limited")
     return ids, gates
+
+
+def moe_bias_update(shape: MoeShape, counts: torch.Tensor, gamma: float,
+                    bias: torch.Tensor) -> torch.Tensor:
+    """bias[e] += gamma * sign(T*k/E - counts[e]), in place; returns bias."""
+    E = shape.experts
+    st = _binding.lib().moe_bias_update(
+        ctypes.byref(shape.c()), _ptr(counts, "counts", torch.int32, (E,)), float(gamma),
+        _ptr(bias, "bias", torch.float32, (E,)), _stream(bias.device))
+    _check(st, "moe_bias_update")
+    return bias
 
 
 def moe_layout(shape: MoeShape, ids: torch.Tensor, *, ws: Workspace,

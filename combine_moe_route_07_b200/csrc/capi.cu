@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cmath>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "moe_route07.h"
@@ -153,6 +155,15 @@ moe_status_t moe_route_limited(const moe_shape_t* shape, const float* logits, co
                                      (shape->flags & MOE_F_RENORM) ? 1 : 0, ids, gates,
                                      static_cast<WsHeader*>(ws), nullptr, 0, R,
                                      max_ranks < R ? max_ranks : 0));
+}
+
+moe_status_t moe_bias_update(const moe_shape_t* shape, const int32_t* counts, float gamma,
+                             float* bias, moe_stream_t stream) {
+  if (!shape_ok(shape) || counts == nullptr || bias == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!std::isfinite(gamma) || gamma < 0.0f) return MOE_ERR_INVALID_ARG;
+  if (!aligned(counts, 4) || !aligned(bias, 4)) return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_bias_update(env_of(stream), counts, shape->experts,
+                                           int64_t(shape->tokens) * shape->k, gamma, bias));
 }
 
 moe_status_t moe_layout(const moe_shape_t* shape, const int32_t* ids, int32_t* counts,

@@ -138,6 +138,10 @@ cudaError_t launch_dispatch_fp8(const LaunchEnv& env, const void* x, const int32
                                 int T, int H, int k, int64_t N, void* out, float* scales,
                                 WsHeader* hdr);
 
+// b_e += gamma * sign(assignments/E - counts[e]) for the E experts, in place.
+cudaError_t launch_bias_update(const LaunchEnv& env, const int32_t* counts, int E,
+                               int64_t assignments, float gamma, float* bias);
+
 // sparse: most slots may be dropped (capacity mode)
 cudaError_t launch_combine(const LaunchEnv& env, const void* y, const int32_t* dst_pos,
                            const float* gates, const void* shared, const void* residual, int T,

@@ -137,6 +137,21 @@ moe_status_t moe_route_limited(const moe_shape_t* shape, const float* logits, co
                                int32_t max_ranks, int32_t* ids, float* gates, void* ws,
                                size_t ws_bytes, moe_stream_t stream);
 
+/* Aux-loss-free balancing: the per-expert bias update from a batch's
+ * histogram ("19. All-to-all", section "Why the router can ruin your day":
+ * a bias per expert bumped up or down based on recent load, used only for the
+ * top-k decision).  For e in [0, E):
+ *   bias[e] += gamma * sign(T*k/E - counts[e])
+ * with the sign taken exactly in integers (an expert exactly at the mean
+ * keeps its bias); one binary32 addition.  The pages give neither gamma nor
+ * the form of the bump; this is the plainest reading.
+ *   counts  int32 [E] assignments per expert (the counts moe_layout writes)
+ *   bias    fp32 [E], updated in place (the bias moe_route takes next)
+ * Both device buffers, 4-byte aligned; gamma finite and >= 0.  Runs on
+ * `stream` after whatever wrote the counts; no workspace. */
+moe_status_t moe_bias_update(const moe_shape_t* shape, const int32_t* counts, float gamma,
+                             float* bias, moe_stream_t stream);
+
 /* Steps 2 and 3 -- count histogram and layout scan ("GPU MoE all-to-all",
  * sections "Two collectives per layer" and "Bucketing"; "MoE All-to-All
  * Dispatch and Ragged Routing", section "Fixed Capacity vs. Ragged Routing").
