@@ -43,6 +43,11 @@ def lib():
         L.orc_layout_src.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp,
                                      vp]
         L.orc_layout_src.restype = i32
+        L.orc_layout_remote_first.argtypes = [i32, i32, i32, i32, i32, i32, i32, vp, vp, vp,
+                                              vp, vp, vp, vp, vp]
+        L.orc_layout_remote_first.restype = i32
+        L.orc_route_round_robin.argtypes = [i32, i32, i32, vp, vp]
+        L.orc_route_round_robin.restype = None
         L.orc_dispatch_bf16.argtypes = [i32, i32, i32, vp, vp, vp]
         L.orc_dispatch_bf16.restype = None
         L.orc_quantize_row_fp8.argtypes = [i32, vp, vp, vp]
@@ -165,6 +170,38 @@ def layout_src(ids, E, R, capacity=0, align=1):
     if rc:
         raise OracleError(f"orc_layout_src status {rc}")
     return out
+
+
+def layout_remote_first(ids, E, R, home, capacity=0, align=1):
+    """Remote-first, tile-aligned layout seen from rank `home`.  Returns the
+    orc_layout dict plus tile_expert [N/align]."""
+    ids = _c(ids, np.int32)
+    T, k = ids.shape
+    N = layout_rows(T, E, k, capacity, align)
+    out = dict(
+        counts=np.empty(E, np.int32),
+        expert_off=np.empty(E + 1, np.int32),
+        rank_off=np.empty(R + 1, np.int32),
+        rank_counts=np.empty(R, np.int32),
+        dst_pos=np.empty((T, k), np.int32),
+        src_idx=np.empty(N, np.int32),
+        tile_expert=np.empty(N // align, np.int32),
+    )
+    rc = lib().orc_layout_remote_first(T, E, k, R, capacity, align, home, _p(ids),
+                                       _p(out["counts"]), _p(out["expert_off"]),
+                                       _p(out["rank_off"]), _p(out["rank_counts"]),
+                                       _p(out["dst_pos"]), _p(out["src_idx"]),
+                                       _p(out["tile_expert"]))
+    if rc:
+        raise OracleError(f"orc_layout_remote_first status {rc}")
+    return out
+
+
+def route_round_robin(T, E, k):
+    ids = np.empty((T, k), np.int32)
+    gates = np.empty((T, k), np.float32)
+    lib().orc_route_round_robin(T, E, k, _p(ids), _p(gates))
+    return ids, gates
 
 
 def dispatch_bf16(x_bits, dst_pos, N):

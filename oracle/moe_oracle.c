@@ -37,6 +37,13 @@
  *   [MSG]  "GPU MoE all-to-all", section "The message-size distribution is
  *          the whole story": an all-to-all over a group of ranks is one
  *          logical message per (sender, receiver) pair, whatever the batch.
+ *   [FIRST] "Mixture-of-experts acceleration through overlap" (thecoregrid):
+ *          remote-owner-aligned layout (each tile bound to one destination
+ *          rank, sent as one contiguous write) and remote-first scheduling
+ *          (the data bound for other GPUs is produced first).
+ *   [DIAG] "GPU MoE all-to-all", section "How to tell whether the
+ *          all-to-all is your bottleneck": replace the learned router by a
+ *          uniform round-robin assignment to separate skew from the wire.
  *   [NODE] "19. All-to-all", opening section: each token is limited to at
  *          most 4 nodes so the slow hop stays bounded; section "Why Qwen3.8's
  *          512 experts is a systems statement": node-limited routing as an
@@ -496,6 +503,93 @@ int orc_layout_src(int T, int E, int k, int R, int capacity, int align, const in
   }
   free(cursor);
   return ORC_OK;
+}
+
+/* Remote-first, tile-aligned layout.  [FIRST], [OWN], [RAG]
+ * As orc_layout, except for the order of the rank slices: seen from rank
+ * `home` (the GPU the batch lives on), the slices of the other ranks come
+ * first, in the order home+1, home+2, ... (mod R), and home's own slice
+ * last.  Experts keep their order inside a slice and assignments their
+ * token order inside an expert.  expert_off[e] is the first row of expert e
+ * (no longer increasing in e); expert_off[E] = rows used; rank_off[r] =
+ * expert_off[r*E/R], rank_off[R] = rows used.  With align = A every expert
+ * segment is a whole number of A-row tiles, each inside one expert and so
+ * bound to one destination rank:
+ *   tile_expert[i]  expert owning rows i*A .. i*A+A-1, -1 past the rows
+ *                   used; N/A entries (N = orc_layout_rows).
+ * In capacity mode the tiles are C rows' worth: A = align = 1 and every row
+ * is a tile. */
+int orc_layout_remote_first(int T, int E, int k, int R, int capacity, int align, int home,
+                            const int32_t* ids, int32_t* counts, int32_t* expert_off,
+                            int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
+                            int32_t* src_idx, int32_t* tile_expert) {
+  if (T < 0 || E < 1 || k < 1 || k > E || R < 1 || E % R != 0 || capacity < 0 || align < 1 ||
+      home < 0 || home >= R)
+    return ORC_BAD_ARG;
+  for (size_t i = 0; i < (size_t)T * k; ++i)
+    if (ids[i] < 0 || ids[i] >= E) return ORC_BAD_ID;
+  const int64_t N = orc_layout_rows(T, E, k, capacity, align);
+  const int Er = E / R;
+
+  for (int e = 0; e < E; ++e) counts[e] = 0;
+  for (size_t i = 0; i < (size_t)T * k; ++i) counts[ids[i]] += 1;
+
+  /* segments in slice order: ranks home+1, ..., home+R (mod R), experts ascending */
+  int32_t run = 0;
+  for (int q = 1; q <= R; ++q) {
+    const int r = (home + q) % R;
+    for (int e = r * Er; e < (r + 1) * Er; ++e) {
+      expert_off[e] = run;
+      run += capacity > 0 ? capacity : ((counts[e] + align - 1) / align) * align;
+    }
+  }
+  expert_off[E] = run;
+  for (int r = 0; r < R; ++r) {
+    rank_off[r] = expert_off[r * Er];
+    int32_t kept = 0;
+    for (int e = r * Er; e < (r + 1) * Er; ++e)
+      kept += (capacity > 0 && counts[e] > capacity) ? capacity : counts[e];
+    rank_counts[r] = kept;
+  }
+  rank_off[R] = expert_off[E];
+
+  for (int64_t p = 0; p < N; ++p) src_idx[p] = -1;
+  int32_t* cursor = (int32_t*)calloc((size_t)E, sizeof(int32_t));
+  if (!cursor) return ORC_BAD_ARG;
+  for (int t = 0; t < T; ++t)
+    for (int j = 0; j < k; ++j) {
+      const size_t i = (size_t)t * k + j;
+      const int e = ids[i];
+      const int32_t c = cursor[e]++;
+      if (capacity > 0 && c >= capacity) {
+        dst_pos[i] = -1;
+        continue;
+      }
+      dst_pos[i] = expert_off[e] + c;
+      src_idx[expert_off[e] + c] = (int32_t)i;
+    }
+  free(cursor);
+
+  /* tile -> expert: walk the segments in slice order */
+  for (int64_t i = 0; i < N / align; ++i) tile_expert[i] = -1;
+  for (int e = 0; e < E; ++e) {
+    const int32_t seg = capacity > 0 ? capacity : ((counts[e] + align - 1) / align) * align;
+    for (int32_t row = expert_off[e]; row < expert_off[e] + seg; row += align)
+      tile_expert[row / align] = e;
+  }
+  return ORC_OK;
+}
+
+/* Round-robin router: the diagnostic that replaces the learned router.
+ * [DIAG]  ids[t,j] = (t*k + j) mod E (k distinct experts per token since
+ * k <= E; every expert gets T*k/E assignments when E divides T*k), gates all
+ * 1/k (rounded to binary32 once). */
+void orc_route_round_robin(int T, int E, int k, int32_t* ids, float* gates) {
+  for (int t = 0; t < T; ++t)
+    for (int j = 0; j < k; ++j) {
+      ids[(size_t)t * k + j] = (int32_t)(((int64_t)t * k + j) % E);
+      gates[(size_t)t * k + j] = (float)(1.0 / (double)k);
+    }
 }
 
 /* ------------------------------------------------------------------------ */
