@@ -28,6 +28,7 @@ from ._binding import MoeError, MOE_F_FP8, MOE_F_RENORM, MOE_F_SRC_LAYOUT
 
 __all__ = ["MoeShape", "Workspace", "Layout", "LayoutSrc", "MoeError", "moe_route", "moe_layout",
            "moe_layout_src", "moe_route_limited", "moe_bias_update",
+           "moe_layout_remote_first", "moe_route_round_robin",
            "moe_route_layout", "moe_route_layout_dispatch",
            "moe_dispatch", "moe_combine", "moe_get_device_error", "moe_check",
            "moe_layout_rows", "moe_workspace_bytes"]
@@ -157,6 +158,50 @@ def moe_route_limited(shape: MoeShape, logits: torch.Tensor, max_ranks: int,
         _ptr(ids, "ids", torch.int32, (T, k)), _ptr(gates, "gates", torch.float32, (T, k)),
         ws.ptr, ws.nbytes, _stream(dev))
     _check(st, "moe_route_limited")
+    return ids, gates
+
+
+def moe_layout_remote_first(shape: MoeShape, ids: torch.Tensor, home_rank: int, *,
+                            ws: Workspace, out: Optional[Layout] = None,
+                            tile_expert: Optional[torch.Tensor] = None):
+    """Layout with the rank slices ordered home+1, ..., home (remote first);
+    returns (Layout, tile_expert int32 [N/align])."""
+    T, E, k, R = shape.tokens, shape.experts, shape.k, shape.ranks
+    N = shape.rows
+    dev = ids.device
+    i32 = dict(dtype=torch.int32, device=dev)
+    if out is None:
+        out = Layout(torch.empty(E, **i32), torch.empty(E + 1, **i32), torch.empty(R + 1, **i32),
+                     torch.empty(R, **i32), torch.empty((T, k), **i32), torch.empty(N, **i32))
+    if tile_expert is None:
+        tile_expert = torch.empty(N // shape.align, **i32)
+    st = _binding.lib().moe_layout_remote_first(
+        ctypes.byref(shape.c()), _ptr(ids, "ids", torch.int32, (T, k)), int(home_rank),
+        _ptr(out.counts, "counts", torch.int32, (E,)),
+        _ptr(out.expert_off, "expert_off", torch.int32, (E + 1,)),
+        _ptr(out.rank_off, "rank_off", torch.int32, (R + 1,)),
+        _ptr(out.rank_counts, "rank_counts", torch.int32, (R,)),
+        _ptr(out.dst_pos, "dst_pos", torch.int32, (T, k)),
+        _ptr(out.src_idx, "src_idx", torch.int32, (N,)),
+        _ptr(tile_expert, "tile_expert", torch.int32, (N // shape.align,)),
+        ws.ptr, ws.nbytes, _stream(dev))
+    _check(st, "moe_layout_remote_first")
+    return out, tile_expert
+
+
+def moe_route_round_robin(shape: MoeShape, *, device=None, ids: Optional[torch.Tensor] = None,
+                          gates: Optional[torch.Tensor] = None):
+    """The round-robin router: ids[t,j] = (t*k + j) mod E, gates 1/k."""
+    T, k = shape.tokens, shape.k
+    dev = device if device is not None else (ids.device if ids is not None else "cuda")
+    if ids is None:
+        ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    if gates is None:
+        gates = torch.empty((T, k), dtype=torch.float32, device=ids.device)
+    st = _binding.lib().moe_route_round_robin(
+        ctypes.byref(shape.c()), _ptr(ids, "ids", torch.int32, (T, k)),
+        _ptr(gates, "gates", torch.float32, (T, k)), _stream(ids.device))
+    _check(st, "moe_route_round_robin")
     return ids, gates
 
 

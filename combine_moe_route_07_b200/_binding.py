@@ -30,7 +30,7 @@ EXPORTS = (
     "moe_workspace_init", "moe_route", "moe_layout", "moe_dispatch", "moe_combine",
     "moe_get_device_error", "moe_layout_noalloc", "moe_route_layout",
     "moe_route_layout_dispatch", "moe_layout_src", "moe_route_limited",
-    "moe_bias_update",
+    "moe_bias_update", "moe_layout_remote_first", "moe_route_round_robin",
 )
 
 
@@ -84,6 +84,10 @@ def lib(path: str = None):
     L.moe_dispatch.restype = i32
     L.moe_combine.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.moe_combine.restype = i32
+    L.moe_layout_remote_first.argtypes = [sp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_layout_remote_first.restype = i32
+    L.moe_route_round_robin.argtypes = [sp, vp, vp, vp]
+    L.moe_route_round_robin.restype = i32
     L.moe_bias_update.argtypes = [sp, vp, ctypes.c_float, vp, vp]
     L.moe_bias_update.restype = i32
     L.moe_route_limited.argtypes = [sp, vp, vp, i32, vp, vp, vp, sz, vp]

@@ -157,6 +157,44 @@ moe_status_t moe_route_limited(const moe_shape_t* shape, const float* logits, co
                                      max_ranks < R ? max_ranks : 0));
 }
 
+moe_status_t moe_layout_remote_first(const moe_shape_t* shape, const int32_t* ids,
+                                     int32_t home_rank, int32_t* counts, int32_t* expert_off,
+                                     int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
+                                     int32_t* src_idx, int32_t* tile_expert, void* ws,
+                                     size_t ws_bytes, moe_stream_t stream) {
+  if (!shape_ok(shape) || src_layout(shape)) return MOE_ERR_INVALID_ARG;
+  if (home_rank < 0 || home_rank >= shape->ranks) return MOE_ERR_INVALID_ARG;
+  const int64_t N = rows_of(shape);
+  if (counts == nullptr || expert_off == nullptr || rank_off == nullptr ||
+      rank_counts == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (shape->tokens > 0 && (ids == nullptr || dst_pos == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (N > 0 && src_idx == nullptr) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {ids, counts, expert_off, rank_off, rank_counts, dst_pos, src_idx,
+                        tile_expert};
+  for (const void* p : ptrs)
+    if (!aligned(p, 4)) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = ws_ok(shape, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  WsHeader* hdr = static_cast<WsHeader*>(ws);
+  uint32_t* tables = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + kHeaderBytes);
+  return from_cuda(moe::launch_layout(env_of(stream), ids, shape->tokens, shape->experts,
+                                      shape->k, shape->ranks, shape->capacity, shape->align, N,
+                                      tables, half_words_of(ws_bytes), hdr, counts, expert_off,
+                                      rank_off, rank_counts, dst_pos, src_idx, true, home_rank,
+                                      tile_expert));
+}
+
+moe_status_t moe_route_round_robin(const moe_shape_t* shape, int32_t* ids, float* gates,
+                                   moe_stream_t stream) {
+  if (!shape_ok(shape)) return MOE_ERR_INVALID_ARG;
+  if (shape->tokens > 0 && (ids == nullptr || gates == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(ids, 4) || !aligned(gates, 4)) return MOE_ERR_INVALID_ARG;
+  if (shape->tokens == 0) return MOE_OK;
+  return from_cuda(moe::launch_route_round_robin(env_of(stream), shape->tokens, shape->experts,
+                                                 shape->k, ids, gates));
+}
+
 moe_status_t moe_bias_update(const moe_shape_t* shape, const int32_t* counts, float gamma,
                              float* bias, moe_stream_t stream) {
   if (!shape_ok(shape) || counts == nullptr || bias == nullptr) return MOE_ERR_INVALID_ARG;

@@ -121,11 +121,15 @@ cudaError_t launch_route(const LaunchEnv& env, const float* logits, const float*
 
 // Layout of `ids` (count pass + place pass).  count_ids == false: the tile
 // table was already filled by a route launch with tables (fused path).
+// 0 <= home < R: rank slices in the order home+1, ..., home (remote first);
+// otherwise the natural order.  tile_expert (or nullptr): the expert of each
+// align-row tile, -1 past the rows used.
 cudaError_t launch_layout(const LaunchEnv& env, const int32_t* ids, int T, int E, int k, int R,
                           int capacity, int align, int64_t N, uint32_t* tables,
                           size_t half_words, WsHeader* hdr, int32_t* counts, int32_t* expert_off,
                           int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
-                          int32_t* src_idx, bool count_ids = true);
+                          int32_t* src_idx, bool count_ids = true, int home = -1,
+                          int32_t* tile_expert = nullptr);
 
 // x_ready: x is not written by the kernel launched just before and every
 // earlier kernel has finished (the case right behind this library's layout
@@ -137,6 +141,10 @@ cudaError_t launch_dispatch_bf16(const LaunchEnv& env, const void* x, const int3
 cudaError_t launch_dispatch_fp8(const LaunchEnv& env, const void* x, const int32_t* dst_pos,
                                 int T, int H, int k, int64_t N, void* out, float* scales,
                                 WsHeader* hdr);
+
+// Round-robin router (diagnostic): ids[t,j] = (t*k + j) mod E, gates 1/k.
+cudaError_t launch_route_round_robin(const LaunchEnv& env, int T, int E, int k, int32_t* ids,
+                                     float* gates);
 
 // b_e += gamma * sign(assignments/E - counts[e]) for the E experts, in place.
 cudaError_t launch_bias_update(const LaunchEnv& env, const int32_t* counts, int E,

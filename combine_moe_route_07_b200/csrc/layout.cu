@@ -79,6 +79,8 @@ __global__ void __launch_bounds__(kCountThreads)
 struct PlaceParams {
   const int32_t* ids;
   int T, k, E, R, capacity, align, G, TT;
+  int home;             // slices in rank order home+1, ..., home (mod R); R-1: natural order
+  int32_t* tile_expert;  // [N/align] expert of each align-row tile, or nullptr
   int staged;
   int64_t N;
   uint32_t* tables;
@@ -134,7 +136,12 @@ __device__ int block_exclusive_scan(int32_t* v, int n, int32_t* warp_tot) {
 }
 
 constexpr size_t place_smem_words(int E, int staged_entries) {
-  return (size_t)(kPlaceThreads / 32) * E + 4 * (size_t)E + 1 + 2 * (size_t)staged_entries;
+  return (size_t)(kPlaceThreads / 32) * E + 5 * (size_t)E + 2 + 2 * (size_t)staged_entries;
+}
+
+// Expert at position q of the slice order (ranks home+1, home+2, ... mod R).
+__device__ __forceinline__ int slice_expert(int q, int home, int R, int Er) {
+  return ((home + 1 + q / Er) % R) * Er + q % Er;
 }
 
 __global__ void __launch_bounds__(kPlaceThreads) place_kernel(const PlaceParams P) {
@@ -146,7 +153,8 @@ __global__ void __launch_bounds__(kPlaceThreads) place_kernel(const PlaceParams 
   int32_t* tot = pre + E;         // [E] total count
   int32_t* off = tot + E;         // [E+1] expert offsets
   int32_t* kept = off + E + 1;    // [E] rows kept per expert
-  int32_t* sid = kept + E;        // [TT*k] staged expert ids
+  int32_t* offq = kept + E;       // [E+1] segment starts in slice order (increasing)
+  int32_t* sid = offq + E + 1;    // [TT*k] staged expert ids
   int32_t* srk = sid + P.TT * k;  // [TT*k] staged ranks inside the warp's run
   __shared__ int32_t s_wtot[kW];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -231,17 +239,26 @@ __global__ void __launch_bounds__(kPlaceThreads) place_kernel(const PlaceParams 
   }
   __syncthreads();
 
-  // 2. expert offsets (every CTA computes the same scan); CTA 0 publishes them
+  // 2. expert offsets (every CTA computes the same scan, in slice order);
+  //    CTA 0 publishes them
+  const int Er = E / P.R;
   for (int e = threadIdx.x; e < E; e += kPlaceThreads) {
     const int c = tot[e];
-    off[e] = C > 0 ? C : ((c + P.align - 1) / P.align) * P.align;
     kept[e] = (C > 0 && c > C) ? C : c;
   }
+  for (int q = threadIdx.x; q < E; q += kPlaceThreads) {
+    const int c = tot[slice_expert(q, P.home, P.R, Er)];
+    offq[q] = C > 0 ? C : ((c + P.align - 1) / P.align) * P.align;
+  }
   __syncthreads();
-  const int used = block_exclusive_scan<kPlaceThreads>(off, E, s_wtot);
-  if (threadIdx.x == 0) off[E] = used;
+  const int used = block_exclusive_scan<kPlaceThreads>(offq, E, s_wtot);
+  for (int q = threadIdx.x; q < E; q += kPlaceThreads) off[slice_expert(q, P.home, P.R, Er)] = offq[q];
+  if (threadIdx.x == 0) {
+    off[E] = used;
+    offq[E] = used;
+  }
+  __syncthreads();
   if (vb == 0) {
-    const int Er = E / P.R;
     for (int e = threadIdx.x; e < E; e += kPlaceThreads) {
       P.counts[e] = tot[e];
       P.expert_off[e] = off[e];
@@ -317,7 +334,7 @@ __global__ void __launch_bounds__(kPlaceThreads) place_kernel(const PlaceParams 
   auto place = [&](int64_t i, int e, int rank) {
     int64_t dst = -1;
     if (rank >= 0)
-      dst = (C > 0) ? (rank < C ? (int64_t)e * C + rank : -1) : (int64_t)off[e] + rank;
+      dst = (C > 0 && rank >= C) ? -1 : (int64_t)off[e] + rank;
     if (dst >= P.N) {  // in range by construction; guards a corrupted tile table
       report(P.hdr, MOE_ERR_DEVICE_RANGE, (int)(dst > INT32_MAX ? INT32_MAX : dst));
       dst = -1;
@@ -336,25 +353,41 @@ __global__ void __launch_bounds__(kPlaceThreads) place_kernel(const PlaceParams 
     run_ranks([&](int64_t i, int e, int v) { place(i, e, v); }, true);  // my[] starts at the bases
   }
 
-  // 5. rows that hold no assignment (alignment padding, unused capacity slots)
+  // 5. rows that hold no assignment (alignment padding, unused capacity
+  //    slots), and the tile map; segments are searched in slice order
+  auto segment_of = [&](int64_t row) {  // last q with offq[q] <= row (row < used)
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (offq[mid] <= row)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    return lo;
+  };
   if (C > 0 || P.align > 1) {
     const int64_t per = (P.N + P.G - 1) / P.G;
     const int64_t r0 = (int64_t)vb * per;
     const int64_t r1 = min(P.N, r0 + per);
     for (int64_t p = r0 + threadIdx.x; p < r1; p += kPlaceThreads) {
       bool pad = true;
-      if (p < off[E]) {
-        int lo = 0, hi = E - 1;  // last e with off[e] <= p
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (off[mid] <= p)
-            lo = mid;
-          else
-            hi = mid - 1;
-        }
-        pad = (p - off[lo]) >= kept[lo];
+      if (p < offq[E]) {
+        const int q = segment_of(p);
+        pad = (p - offq[q]) >= kept[slice_expert(q, P.home, P.R, Er)];
       }
       if (pad) P.src_idx[p] = -1;
+    }
+  }
+  if (P.tile_expert != nullptr) {
+    const int64_t ntiles = P.N / P.align;
+    const int64_t per = (ntiles + P.G - 1) / P.G;
+    const int64_t a0 = (int64_t)vb * per;
+    const int64_t a1 = min(ntiles, a0 + per);
+    for (int64_t i = a0 + threadIdx.x; i < a1; i += kPlaceThreads) {
+      const int64_t row = i * P.align;
+      P.tile_expert[i] =
+          row < offq[E] ? slice_expert(segment_of(row), P.home, P.R, Er) : -1;
     }
   }
 
@@ -382,7 +415,7 @@ cudaError_t launch_layout(const LaunchEnv& env, const int32_t* ids, int T, int E
                           int capacity, int align, int64_t N, uint32_t* tables,
                           size_t half_words, WsHeader* hdr, int32_t* counts, int32_t* expert_off,
                           int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
-                          int32_t* src_idx, bool count_ids) {
+                          int32_t* src_idx, bool count_ids, int home, int32_t* tile_expert) {
   const TileGeom geom = layout_tiles(T);
   cudaError_t err;
   if (count_ids && T > 0) {
@@ -405,6 +438,8 @@ cudaError_t launch_layout(const LaunchEnv& env, const int32_t* ids, int T, int E
   P.R = R;
   P.capacity = capacity;
   P.align = align;
+  P.home = (home >= 0 && home < R) ? home : R - 1;
+  P.tile_expert = tile_expert;
   P.G = geom.G;
   P.TT = geom.TT;
   P.N = N;

@@ -206,7 +206,35 @@ cudaError_t launch_any(const LaunchEnv& env, const float* logits, const float* b
                              table_words, R, M);
 }
 
+// The round-robin router: ids[t,j] = (t*k + j) mod E, gates 1/k.  "GPU MoE
+// all-to-all", section "How to tell whether the all-to-all is your
+// bottleneck": swapping the learned router for a uniform round-robin
+// assignment separates routing skew from the cost of the exchange itself.
+__global__ void __launch_bounds__(kThreads)
+    round_robin_kernel(int T, int E, int k, int32_t* __restrict__ ids,
+                       float* __restrict__ gates) {
+  pdl_wait();  // ids and gates may still be read by the kernel launched before
+  pdl_trigger();
+  const int64_t n = (int64_t)T * k;
+  const float g = (float)(1.0 / (double)k);
+  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * kThreads) {
+    ids[i] = (int32_t)(i % E);  // i = t*k + j
+    gates[i] = g;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_route_round_robin(const LaunchEnv& env, int T, int E, int k, int32_t* ids,
+                                     float* gates) {
+  const int64_t n = (int64_t)T * k;
+  int64_t grid = (n + kThreads - 1) / kThreads;
+  if (grid > 4 * (int64_t)env.num_sms) grid = 4 * (int64_t)env.num_sms;
+  if (grid < 1) grid = 1;
+  return launch_pdl(env, round_robin_kernel, dim3((unsigned)grid), dim3(kThreads), 0, T, E, k,
+                    ids, gates);
+}
 
 cudaError_t launch_route(const LaunchEnv& env, const float* logits, const float* bias, int T,
                          int E, int k, int renorm, int32_t* ids, float* gates, WsHeader* hdr,

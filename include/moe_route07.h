@@ -137,6 +137,37 @@ moe_status_t moe_route_limited(const moe_shape_t* shape, const float* logits, co
                                int32_t max_ranks, int32_t* ids, float* gates, void* ws,
                                size_t ws_bytes, moe_stream_t stream);
 
+/* Remote-first, tile-aligned layout ("Mixture-of-experts acceleration
+ * through overlap": a remote-owner-aligned layout where every tile belongs to
+ * one destination rank and is written contiguously, and remote-first
+ * scheduling: the data bound for other GPUs is produced first).  Same outputs
+ * and rules as moe_layout, except that the rank slices are ordered as seen
+ * from rank `home_rank` (the GPU holding the batch): home+1, home+2, ...
+ * (mod R), and home's own slice last.  expert_off[e] is then the first row of
+ * expert e (not increasing in e); rank_off[r] = expert_off[r*E/R] and
+ * rank_off[R] = rows used.  With align = A (the grouped-GEMM tile height,
+ * e.g. 128) every expert segment is a whole number of A-row tiles:
+ *   tile_expert  int32 [N/A] expert owning rows i*A .. i*A+A-1, -1 past the
+ *                rows used (NULL: not written)
+ * 0 <= home_rank < R, else MOE_ERR_INVALID_ARG; home_rank = R-1 gives exactly
+ * moe_layout.  The pages give no order among the remote slices; the rotation
+ * is the usual all-to-all schedule. */
+moe_status_t moe_layout_remote_first(const moe_shape_t* shape, const int32_t* ids,
+                                     int32_t home_rank, int32_t* counts, int32_t* expert_off,
+                                     int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
+                                     int32_t* src_idx, int32_t* tile_expert, void* ws,
+                                     size_t ws_bytes, moe_stream_t stream);
+
+/* The round-robin router, a diagnostic ("GPU MoE all-to-all", section "How
+ * to tell whether the all-to-all is your bottleneck": replace the learned
+ * router by a uniform round-robin assignment; a much faster exchange means
+ * the problem is skew, not the wire):
+ *   ids[t,j] = (t*k + j) mod E,  gates[t,j] = 1/k (rounded once to fp32)
+ * k distinct experts per token; every expert gets T*k/E assignments when E
+ * divides T*k.  Buffers as moe_route; no workspace. */
+moe_status_t moe_route_round_robin(const moe_shape_t* shape, int32_t* ids, float* gates,
+                                   moe_stream_t stream);
+
 /* Aux-loss-free balancing: the per-expert bias update from a batch's
  * histogram ("19. All-to-all", section "Why the router can ruin your day":
  * a bias per expert bumped up or down based on recent load, used only for the
