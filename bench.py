@@ -57,6 +57,13 @@ def parse():
                    help="> 0: each step also runs the aux-loss-free bias update "
                         "(moe_bias_update) with this step size; the bias feeds the next step's "
                         "route")
+    p.add_argument("--router", choices=["learned", "round_robin"], default="learned",
+                   help="round_robin: the diagnostic router (ids (t*k+j) mod E, gates 1/k) in "
+                        "place of the learned one")
+    p.add_argument("--home", type=int, default=-1,
+                   help=">= 0: remote-first layout seen from this rank (moe_layout_remote_first)")
+    p.add_argument("--align", type=int, default=0,
+                   help="> 0: override the workload's segment alignment (e.g. 128-row tiles)")
     p.add_argument("--tokens", type=int, default=0,
                    help="override the workload's token count (smaller cases for profiler "
                         "captures; a changed workload, not a bench line)")
@@ -78,7 +85,9 @@ def algorithmic_bytes(w, kept_rows):
     b["route"] = T * E * 4 + (4 * E if w.bias else 0) + T * k * 8
     b["route_limited"] = b["route"]
     b["bias_update"] = 12 * E  # counts in, bias in and out
+    b["route_round_robin"] = T * k * 8  # ids and gates out
     b["layout"] = T * k * 4 * 2 + w.rows * 4 + (3 * E + 2 * w.R) * 4  # ids in, dst_pos/src_idx out
+    b["layout_remote_first"] = b["layout"] + (w.rows // w.align) * 4  # + the tile map
     b["dispatch"] = T * row + kept_rows * disp_row_out + T * k * 4
     b["combine"] = kept_rows * row + T * k * 8 + T * row \
         + (T * row if w.shared else 0) + (T * row if w.residual else 0)
@@ -302,6 +311,8 @@ def main():
     w = WORKLOADS[args.workload]
     if args.tokens > 0:
         w = w.with_(name=f"{w.name}_t{args.tokens}", T=args.tokens)
+    if args.align > 0:
+        w = w.with_(name=f"{w.name}_a{args.align}", align=args.align)
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -359,32 +370,40 @@ def main():
 
     M = args.max_ranks
 
+    RR = args.router == "round_robin"
+    HOME = args.home
+
     def route_op():
-        if M > 0:
+        if RR:
+            m.moe_route_round_robin(shape, ids=ids, gates=gates)
+        elif M > 0:
             m.moe_route_limited(shape, logits, M, bias, ws=ws, ids=ids, gates=gates)
         else:
             m.moe_route(shape, logits, bias, ws=ws, ids=ids, gates=gates)
 
-    def route_layout_dispatch():
-        route_op()
+    tile_expert = (torch.empty(N // w.align, dtype=torch.int32, device=dev) if HOME >= 0
+                   else None)
+
+    def layout_op():
         if src:
             m.moe_layout_src(shape, ids, ws=ws, out=lay)
+        elif HOME >= 0:
+            m.moe_layout_remote_first(shape, ids, HOME, ws=ws, out=lay, tile_expert=tile_expert)
         else:
             m.moe_layout(shape, ids, ws=ws, out=lay)
+
+    def route_layout_dispatch():
+        route_op()
+        layout_op()
         m.moe_dispatch(shape, x, lay.dst_pos, ws=ws, out=xd, scales=sc)
 
     # the expert stand-in's output for this batch, prepared once
     route_layout_dispatch()
     if w.fp8:
         y = (xd.float() * sc.repeat_interleave(128, dim=1)).to(torch.bfloat16)
-    elif w.expert == "scale" and src:
-        e = ids.flatten()[lay.src_idx.clamp(min=0).long()].long()
-        s = (torch.arange(1, w.E + 1, dtype=torch.float32, device=dev)
-             / torch.tensor(float(w.E), device=dev))[e]
-        y = (xd.float() * s[:, None]).to(torch.bfloat16)
     elif w.expert == "scale":
-        rows = torch.arange(N, device=dev, dtype=torch.int32)
-        e = (torch.searchsorted(lay.expert_off, rows, right=True) - 1).clamp(min=0)
+        # expert of every row from src_idx (any row order); empty rows read expert 0
+        e = ids.flatten()[lay.src_idx.clamp(min=0).long()].long()
         s = (torch.arange(1, w.E + 1, dtype=torch.float32, device=dev)
              / torch.tensor(float(w.E), device=dev))[e]
         y = (xd.float() * s[:, None]).to(torch.bfloat16)
@@ -418,13 +437,13 @@ def main():
     if G > 0:
         names_probe = ("route_layout", "dispatch", "bias_update", "combine")
         ops_probe = (ops_probe[0], ops_probe[1], bias_op, ops_probe[2])
-    if src or M > 0:
-        names = ("route_limited" if M > 0 else "route", "layout_src" if src else "layout",
+    if src or M > 0 or RR or HOME >= 0:
+        names = ("route_round_robin" if RR else ("route_limited" if M > 0 else "route"),
+                 "layout_src" if src else ("layout_remote_first" if HOME >= 0 else "layout"),
                  "dispatch", "combine")
         ops = (
             route_op,
-            (lambda: m.moe_layout_src(shape, ids, ws=ws, out=lay)) if src else
-            (lambda: m.moe_layout(shape, ids, ws=ws, out=lay)),
+            layout_op,
             lambda: m.moe_dispatch(shape, x, lay.dst_pos, ws=ws, out=xd, scales=sc),
             lambda: m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared,
                                   residual=residual, out=out),
@@ -509,7 +528,7 @@ def main():
     # per-kernel breakdown: a probe graph of the same step with event-record
     # nodes between the kernels, replayed after an L2 flush and read back one
     # replay at a time
-    separate = src or M > 0
+    separate = src or M > 0 or RR or HOME >= 0
     probe_names = names if (separate or args.path != "fused3") else names_probe
     probe_ops = ops if (separate or args.path != "fused3") else ops_probe
     n_ops = len(probe_ops)
@@ -627,6 +646,8 @@ def main():
                              "rows by expert, token",
                    "max_ranks": M if M > 0 else None,
                    "bias_gamma": G if G > 0 else None,
+                   "router": args.router,
+                   "home_rank": HOME if HOME >= 0 else None,
                    "step": " + ".join(names) + ", one CUDA graph"},
         "dispatch_combine": {"tokens_per_s": world * T / (dc_ms * 1e-3),
                              "us": round(dc_ms * 1e3, 2), "gbs": round(dc_gbs, 1),

@@ -72,3 +72,17 @@ def test_reference_arm_prints_one_line_and_other_ranks_stay_silent(capsys, monke
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_algorithmic_bytes_cover_every_step_name():
+    """Every kernel name a bench path can report has a byte count."""
+    import bench
+    from combine_moe_route_07_b200.workloads import WORKLOADS
+    names = {"route", "route_limited", "route_round_robin", "layout", "layout_src",
+             "layout_remote_first", "dispatch", "combine", "bias_update", "route_layout",
+             "route_layout_dispatch"}
+    for w in WORKLOADS.values():
+        for ww in (w, w.with_(align=128) if not w.capacity else w):
+            b = bench.algorithmic_bytes(ww, ww.rows)
+            assert names <= set(b), names - set(b)
+            assert all(v > 0 for v in b.values())
