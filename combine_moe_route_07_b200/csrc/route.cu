@@ -27,14 +27,14 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;  // tokens per CTA group
 constexpr uint64_t kRowTimeoutNs = 1000000000ull;
 
-template <int NK, bool HIST, bool STAGE>
+template <int NK, bool HIST, bool STAGE, bool LIMIT>
 __global__ void __launch_bounds__(kThreads)
     route_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E,
                  int k, int renorm, int32_t* __restrict__ ids, float* __restrict__ gates,
                  WsHeader* hdr, uint32_t* __restrict__ tables, int TT, size_t table_words,
                  int per, int R, int M) {
   // dynamic: [hist: E int32, padded to 16 B] (HIST), [rows: kWarps x 2 x E floats] (STAGE),
-  // [rank limit: kWarps x (R + ceil(R/32)) words] (M < R)
+  // [rank limit: kWarps x (R + ceil(R/32)) words] (M < R), [bias: E floats] (STAGE)
   extern __shared__ __align__(16) unsigned char dyn[];
   __shared__ uint32_t cand_all[kWarps][NK >= 8 ? 3 * kMaxCand : 1];
   __shared__ uint64_t bars[kWarps][2];
@@ -42,16 +42,15 @@ __global__ void __launch_bounds__(kThreads)
   const size_t hist_bytes = HIST ? (((size_t)E * 4 + 15) & ~(size_t)15) : 0;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   float* buf = reinterpret_cast<float*>(dyn + hist_bytes) + (size_t)w * 2 * E;
-  RankLimit lim;
+  RankLimit lim;  // compiled in only for LIMIT (then M < R)
   lim.R = R;
-  lim.M = M;
+  lim.M = LIMIT ? M : 0;
   lim.init(E, lane);
-  if (lim.on()) {
-    const size_t lim_words = (size_t)R + (R + 31) / 32;
-    lim.smem = reinterpret_cast<uint32_t*>(dyn + hist_bytes +
-                                           (STAGE ? (size_t)kWarps * 2 * E * sizeof(float) : 0)) +
-               (size_t)w * lim_words;
-  }
+  const size_t lim_words = lim.on() ? (size_t)R + (R + 31) / 32 : 0;
+  uint32_t* lim_base = reinterpret_cast<uint32_t*>(
+      dyn + hist_bytes + (STAGE ? (size_t)kWarps * 2 * E * sizeof(float) : 0));
+  if (lim.on()) lim.smem = lim_base + (size_t)w * lim_words;
+  float* sbias = reinterpret_cast<float*>(lim_base + (size_t)kWarps * lim_words);
   if (STAGE && lane == 0) {
     mbar_init(&bars[w][0], 1);
     mbar_init(&bars[w][1], 1);
@@ -61,7 +60,11 @@ __global__ void __launch_bounds__(kThreads)
   pdl_wait();  // logits (and the tile table) may come from the kernel launched before
   pdl_trigger();
   float b[NK];
-  load_bias<NK>(bias, E, lane, b);
+  if constexpr (!STAGE) load_bias<NK>(bias, E, lane, b);
+  if constexpr (STAGE) {  // the bias, read per token from shared memory
+    for (int e = threadIdx.x; e < E; e += kThreads) sbias[e] = bias != nullptr ? __ldg(bias + e) : 0.0f;
+    __syncthreads();
+  }
   const int c0 = (int)min((int64_t)blockIdx.x * per, (int64_t)T);
   const int c1 = min(T, c0 + per);
   const int n = (c1 - c0 + kWarps - 1) / kWarps;  // groups: the same for every warp
@@ -121,8 +124,8 @@ __global__ void __launch_bounds__(kThreads)
         if (ok) {
           parity ^= 1u << sb;
           pending &= ~(1u << sb);
-          nan_tok = route_token_thr<NK, true>(logits, t, T, b, E, k, renorm, lane, cand_all[w],
-                                              e1, g1, buf + (size_t)sb * E, lim);
+          nan_tok = route_token_smem<NK, LIMIT>(buf + (size_t)sb * E, sbias, t, E, k, renorm,
+                                                lane, cand_all[w], e1, g1, lim);
         } else {
           if (lane == 0) report(hdr, MOE_ERR_DEVICE_TIMEOUT, t);
           alive = false;  // routes nothing more; still takes part in the CTA barriers
@@ -166,10 +169,14 @@ cudaError_t launch_nk(const LaunchEnv& env, const float* logits, const float* bi
   const size_t hist_bytes = HIST ? (((size_t)E * 4 + 15) & ~(size_t)15) : 0;
   // rows staged by bulk copy: many keys per lane, 16-byte rows and base
   const bool stage = NK >= 8 && (E % 4) == 0 && (reinterpret_cast<uintptr_t>(logits) & 15u) == 0;
-  auto kern = stage ? route_kernel<NK, HIST, NK >= 8> : route_kernel<NK, HIST, false>;
   const bool limit = M > 0 && M < R;
+  auto kern = stage ? (limit ? route_kernel<NK, HIST, NK >= 8, true>
+                             : route_kernel<NK, HIST, NK >= 8, false>)
+                    : (limit ? route_kernel<NK, HIST, false, true>
+                             : route_kernel<NK, HIST, false, false>);
   const size_t smem = hist_bytes + (stage ? (size_t)kWarps * 2 * E * sizeof(float) : 0) +
-                      (limit ? (size_t)kWarps * (R + (R + 31) / 32) * sizeof(uint32_t) : 0);
+                      (limit ? (size_t)kWarps * (R + (R + 31) / 32) * sizeof(uint32_t) : 0) +
+                      (stage ? (size_t)E * sizeof(float) : 0);
   int per_sm = 1;
   const cudaError_t err = blocks_per_sm(reinterpret_cast<const void*>(kern), kThreads, smem, &per_sm);
   if (err != cudaSuccess) return err;

@@ -435,4 +435,136 @@ __device__ __forceinline__ int route_token_thr(const float* __restrict__ logits,
   return nan_tok;
 }
 
+// Threshold top-k for a token whose logits row (and the bias) sit in shared
+// memory: only the key codes live in registers, the raw logits are re-read
+// from the row where they are needed (the candidates, the winner of a full
+// scan, the full softmax without renorm).  The same decisions as
+// route_token_thr: tau = the k-th largest lane maximum, compaction of the
+// keys >= tau, k rounds over at most two candidates per lane; more than
+// kMaxCand candidates (heavy ties) takes k rounds over all the codes.
+template <int NK, bool LIMIT>
+__device__ __forceinline__ int route_token_smem(const float* srow, const float* sbias, int t,
+                                                int E, int k, int renorm, int lane,
+                                                uint32_t* cand, int& sel_e, float& gate,
+                                                const RankLimit& lim) {
+  uint32_t code[NK];
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < NK; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E) {
+      const float key = __fadd_rn(srow[e], sbias[e]);
+      bad |= (key != key);
+      code[i] = order_code(key);
+    } else {
+      code[i] = 0u;
+    }
+  }
+  const int nan_tok = __any_sync(kFull, bad) ? t : -1;
+  if constexpr (LIMIT) apply_rank_limit<NK>(code, E, lane, lim);
+
+  uint32_t mm = 0u;
+#pragma unroll
+  for (int i = 0; i < NK; ++i) mm = max(mm, code[i]);
+  uint32_t tau = 0u;
+  for (int j = 0; j < k; ++j) {
+    const uint32_t top = __reduce_max_sync(kFull, mm);
+    tau = top;
+    const unsigned hold = __ballot_sync(kFull, mm == top);
+    if (lane == __ffs(hold) - 1) mm = 0u;
+  }
+  int c = 0;
+#pragma unroll
+  for (int i = 0; i < NK; ++i) c += (code[i] != 0u && code[i] >= tau) ? 1 : 0;
+  const int total = (int)__reduce_add_sync(kFull, (unsigned)c);
+
+  float sel_raw = 0.0f;
+  sel_e = 0;
+  if (total > kMaxCand) {  // heavy ties at the threshold: k rounds over every code
+    for (int j = 0; j < k; ++j) {
+      uint32_t best = 0u;
+      int bi = 0;
+#pragma unroll
+      for (int i = 0; i < NK; ++i)
+        if (code[i] > best) {  // strict: the lowest index wins ties
+          best = code[i];
+          bi = i;
+        }
+      const uint32_t top = __reduce_max_sync(kFull, best);
+      const uint32_t win =
+          __reduce_min_sync(kFull, (best == top) ? (uint32_t)(lane + 32 * bi) : 0xffffffffu);
+#pragma unroll
+      for (int i = 0; i < NK; ++i)
+        if ((uint32_t)(lane + 32 * i) == win) code[i] = 0u;
+      if (lane == j) {
+        sel_e = (int)win;
+        sel_raw = srow[win];
+      }
+    }
+  } else {
+    int pre = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, pre, o);
+      if (lane >= o) pre += y;
+    }
+    pre -= c;
+#pragma unroll
+    for (int i = 0; i < NK; ++i)
+      if (code[i] != 0u && code[i] >= tau) {
+        cand[pre] = code[i];
+        cand[kMaxCand + pre] = (uint32_t)(lane + 32 * i);
+        ++pre;
+      }
+    __syncwarp();
+    uint32_t c0 = 0u, c1 = 0u, e0 = 0u, e1 = 0u;
+    if (lane < total) {
+      c0 = cand[lane];
+      e0 = cand[kMaxCand + lane];
+    }
+    if (lane + 32 < total) {
+      c1 = cand[lane + 32];
+      e1 = cand[kMaxCand + lane + 32];
+    }
+    __syncwarp();  // the next token may overwrite cand
+    for (int j = 0; j < k; ++j) {
+      const bool use1 = (c1 > c0) || (c1 == c0 && c1 != 0u && e1 < e0);
+      const uint32_t bk = use1 ? c1 : c0;
+      const uint32_t be = use1 ? e1 : e0;
+      const uint32_t top = __reduce_max_sync(kFull, bk);
+      const uint32_t win = __reduce_min_sync(kFull, (bk == top) ? be : 0xffffffffu);
+      if (bk == top && be == win) {
+        if (use1)
+          c1 = 0u;
+        else
+          c0 = 0u;
+      }
+      if (lane == j) {
+        sel_e = (int)win;
+        sel_raw = srow[win];
+      }
+    }
+  }
+
+  if (renorm) {
+    const float m = warp_max_f(lane < k ? sel_raw : -INFINITY);
+    const double ex = (lane < k) ? exp((double)sel_raw - (double)m) : 0.0;
+    const double den = warp_sum_d(ex);
+    gate = (float)(ex / den);
+  } else {
+    float lm = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < NK; ++i)
+      if (lane + 32 * i < E) lm = fmaxf(lm, srow[lane + 32 * i]);
+    const float m = warp_max_f(lm);
+    double part = 0.0;
+#pragma unroll
+    for (int i = 0; i < NK; ++i)
+      if (lane + 32 * i < E) part += exp((double)srow[lane + 32 * i] - (double)m);
+    const double den = warp_sum_d(part);
+    gate = (float)(exp((double)sel_raw - (double)m) / den);
+  }
+  return nan_tok;
+}
+
 }  // namespace moe
