@@ -68,14 +68,20 @@ struct RankLimit {
   int step = 0;  // mode 1: ranks per column; mode 2: columns per rank
   int lane_rank = 0;
   bool lead = false;
+  bool col_map = false;  // Er divides 32: key i of this lane is on rank i * step + lane_rank
+  uint32_t magic = 0u;   // Er >= 2: ceil(2^32 / Er), n / Er == __umulhi(n, magic) for n < 2^16
   __device__ bool on() const { return M > 0 && M < R; }
   __device__ void init(int E, int lane) {
     Er = E / R;
-    if (Er <= 32 && (32 % Er) == 0 && R <= 64) {
-      mode = 1;
+    magic = Er >= 2 ? (uint32_t)((0x100000000ull + (uint64_t)Er - 1) / (uint64_t)Er) : 0u;
+    col_map = Er <= 32 && (32 % Er) == 0;
+    if (col_map) {
       step = 32 / Er;
       lane_rank = lane / Er;
       lead = (lane % Er) == 0;
+    }
+    if (col_map && R <= 64) {
+      mode = 1;
     } else if ((Er & 31) == 0) {
       mode = 2;
       step = Er >> 5;
@@ -435,6 +441,70 @@ __device__ __forceinline__ int route_token_thr(const float* __restrict__ logits,
   return nan_tok;
 }
 
+// Rank limit for a token whose row and bias sit in shared memory, decided
+// before any key code is formed: lane l scores ranks l, l+32, ... straight
+// from the row (the largest key code over the rank's experts) and M rounds of
+// a warp arg-max pick the kept ranks.  R <= 64: returns the kept ranks as a
+// 64-bit mask; larger R: marks them in this warp's shared bitmap (L.smem + R)
+// and returns 0.
+__device__ __forceinline__ uint64_t rank_limit_smem(const float* srow, const float* sbias,
+                                                    int lane, const RankLimit& L) {
+  const int R = L.R, Er = L.Er;
+  auto score = [&](int r) {
+    uint32_t best = 0u;
+    for (int e = r * Er; e < (r + 1) * Er; ++e)
+      best = max(best, order_code(__fadd_rn(srow[e], sbias[e])));
+    return best;
+  };
+  if (R <= 64) {
+    const uint32_t s0 = lane < R ? score(lane) : 0u;
+    const uint32_t s1 = lane + 32 < R ? score(lane + 32) : 0u;
+    uint64_t kept = 0ull;
+    for (int m = 0; m < L.M; ++m) {
+      const uint32_t b0 = ((kept >> lane) & 1ull) ? 0u : s0;  // valid scores are never 0
+      const uint32_t b1 = ((kept >> (lane + 32)) & 1ull) ? 0u : s1;
+      const uint32_t best = max(b0, b1);
+      const uint32_t id = b0 >= b1 ? (uint32_t)lane : (uint32_t)(lane + 32);
+      const uint32_t top = __reduce_max_sync(kFull, best);
+      kept |= 1ull << __reduce_min_sync(kFull, best == top ? id : 0xffffffffu);
+    }
+    return kept;
+  }
+  uint32_t* rmax = L.smem;
+  uint32_t* chosen = L.smem + R;
+  __syncwarp();  // the previous token is done with the words
+  for (int r = lane; r < R; r += 32) rmax[r] = score(r);
+  for (int q = lane; q < (R + 31) / 32; q += 32) chosen[q] = 0u;
+  __syncwarp();
+  for (int m = 0; m < L.M; ++m) {
+    uint32_t best = 0u;
+    int bi = R;
+    for (int r = lane; r < R; r += 32) {  // ascending r: strict > keeps the lower id
+      if (((chosen[r >> 5] >> (r & 31)) & 1u) == 0u) {
+        const uint32_t v = rmax[r];
+        if (bi == R || v > best) {
+          best = v;
+          bi = r;
+        }
+      }
+    }
+    const uint32_t top = __reduce_max_sync(kFull, best);
+    const uint32_t win =
+        __reduce_min_sync(kFull, (bi < R && best == top) ? (uint32_t)bi : 0xffffffffu);
+    if (lane == 0) chosen[win >> 5] |= 1u << (win & 31u);
+    __syncwarp();
+  }
+  return 0ull;
+}
+
+// Is the rank of expert e kept?  (the mask or bitmap rank_limit_smem made)
+__device__ __forceinline__ bool rank_kept(int e, int i, int lane, uint64_t kept,
+                                          const RankLimit& L) {
+  const int r = L.col_map ? i * L.step + L.lane_rank : (int)__umulhi((uint32_t)e, L.magic);
+  if (L.R <= 64) return ((kept >> r) & 1ull) != 0ull;
+  return ((L.smem[L.R + (r >> 5)] >> (r & 31)) & 1u) != 0u;
+}
+
 // Threshold top-k for a token whose logits row (and the bias) sit in shared
 // memory: only the key codes live in registers, the raw logits are re-read
 // from the row where they are needed (the candidates, the winner of a full
@@ -447,6 +517,8 @@ __device__ __forceinline__ int route_token_smem(const float* srow, const float* 
                                                 int E, int k, int renorm, int lane,
                                                 uint32_t* cand, int& sel_e, float& gate,
                                                 const RankLimit& lim) {
+  uint64_t kept = 0ull;
+  if constexpr (LIMIT) kept = rank_limit_smem(srow, sbias, lane, lim);
   uint32_t code[NK];
   bool bad = false;
 #pragma unroll
@@ -456,12 +528,13 @@ __device__ __forceinline__ int route_token_smem(const float* srow, const float* 
       const float key = __fadd_rn(srow[e], sbias[e]);
       bad |= (key != key);
       code[i] = order_code(key);
+      if constexpr (LIMIT)
+        if (!rank_kept(e, i, lane, kept, lim)) code[i] = 0u;
     } else {
       code[i] = 0u;
     }
   }
   const int nan_tok = __any_sync(kFull, bad) ? t : -1;
-  if constexpr (LIMIT) apply_rank_limit<NK>(code, E, lane, lim);
 
   uint32_t mm = 0u;
 #pragma unroll
