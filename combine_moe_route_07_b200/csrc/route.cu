@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(kThreads)
         }
       } else if constexpr (NK >= 8) {
         nan_tok = route_token_thr<NK>(logits, t, T, b, E, k, renorm, lane, cand_all[w], e1, g1,
-                                      nullptr, lim);
+                                      lim);
       } else {
         int tok[1] = {t}, ea[1];
         float ga[1];

@@ -8,10 +8,14 @@
 // Lane l holds experts l, l+32, l+64, ... of each token in registers, as
 // order-preserving 32-bit codes of key = logit + bias.  Each of the k rounds
 // is two hardware warp reductions (redux.sync): the largest code, then the
-// lowest expert id among the lanes holding it, which is the tie rule.  TPW
-// tokens go through the rounds together so their latency chains overlap.
-// The gates are a softmax of the selected RAW logits evaluated in fp64 (k
-// values per token) and rounded to fp32 once.
+// lowest expert id among the lanes holding it, which is the tie rule.  Three
+// forms of the same selection: route_tokens (every code, k rounds; E <= 224),
+// route_token_thr (a threshold first, then the rounds over the few keys
+// above it) and route_token_smem (the threshold form with the row and the
+// bias read from shared memory, only the codes in registers).  An optional
+// rank limit clears the codes of all but the M best ranks first.  The gates
+// are a softmax of the selected RAW logits evaluated in fp64 (k values per
+// token) and rounded to fp32 once.
 #pragma once
 
 #include <math.h>
@@ -206,12 +210,6 @@ __device__ __forceinline__ void apply_rank_limit(uint32_t (&code)[NK], int E, in
   __syncwarp();  // the next token reuses the words
 }
 
-// Tokens per warp group for NK keys per lane (register budget).
-template <int NK>
-struct RouteGroup {
-  static constexpr int value = NK <= 4 ? 4 : (NK <= 8 ? 2 : 1);
-};
-
 // Route tokens tok[0..TPW) (entries >= T are skipped).  On return lane j < k
 // holds slot j of token u: expert sel_e[u], gate[u].  Returns the first token
 // with a NaN key, or -1.
@@ -310,17 +308,15 @@ __device__ __forceinline__ int route_tokens(const float* __restrict__ logits, co
 // selected.  The warp compacts the keys >= tau (usually k to 2k of them) into
 // shared memory and runs the k selection rounds over at most two per lane.
 // More than kMaxCand candidates (heavy ties) falls back to route_tokens.
-// `cand` is this warp's 3*kMaxCand words of shared memory.  With SMEM the
-// token's logits are read from `srow` (a copy of the row in shared memory)
-// instead of from global memory.
+// `cand` is this warp's 3*kMaxCand words of shared memory.  (Rows staged in
+// shared memory go through route_token_smem instead.)
 constexpr int kMaxCand = 64;
 
-template <int NK, bool SMEM = false>
+template <int NK>
 __device__ __forceinline__ int route_token_thr(const float* __restrict__ logits, int t, int T,
                                                const float (&b)[NK], int E, int k, int renorm,
                                                int lane, uint32_t* cand, int& sel_e,
-                                               float& gate, const float* srow = nullptr,
-                                               const RankLimit& lim = RankLimit()) {
+                                               float& gate, const RankLimit& lim = RankLimit()) {
   float raw[NK];
   uint32_t code[NK];
   bool bad = false;
@@ -329,7 +325,7 @@ __device__ __forceinline__ int route_token_thr(const float* __restrict__ logits,
   for (int i = 0; i < NK; ++i) {
     const int e = lane + 32 * i;
     if (e < E) {
-      raw[i] = SMEM ? srow[e] : __ldcs(row + e);
+      raw[i] = __ldcs(row + e);
       const float key = __fadd_rn(raw[i], b[i]);
       bad |= (key != key);
       code[i] = order_code(key);
