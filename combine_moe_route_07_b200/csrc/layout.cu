@@ -40,7 +40,7 @@ namespace {
 constexpr int kCountThreads = 256;
 constexpr int kPlaceThreads = 512;
 constexpr int kUnroll = 4;
-constexpr int kMaxStaged = 4096;  // assignments per tile kept in smem across the passes
+constexpr int kMaxStaged = 8192;  // assignments per tile kept in smem across the passes
 constexpr int kRowsInFlight = 8;  // tile rows each warp loads before adding
 
 __global__ void __launch_bounds__(kCountThreads)
