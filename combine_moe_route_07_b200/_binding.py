@@ -31,6 +31,7 @@ EXPORTS = (
     "moe_get_device_error", "moe_layout_noalloc", "moe_route_layout",
     "moe_route_layout_dispatch", "moe_layout_src", "moe_route_limited",
     "moe_bias_update", "moe_layout_remote_first", "moe_route_round_robin",
+    "moe_selftest_wait_timeout",
 )
 
 
@@ -88,6 +89,8 @@ def lib(path: str = None):
     L.moe_layout_remote_first.restype = i32
     L.moe_route_round_robin.argtypes = [sp, vp, vp, vp]
     L.moe_route_round_robin.restype = i32
+    L.moe_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint32, vp]
+    L.moe_selftest_wait_timeout.restype = i32
     L.moe_bias_update.argtypes = [sp, vp, ctypes.c_float, vp, vp]
     L.moe_bias_update.restype = i32
     L.moe_route_limited.argtypes = [sp, vp, vp, i32, vp, vp, vp, sz, vp]

@@ -357,6 +357,13 @@ moe_status_t moe_combine(const moe_shape_t* shape, const void* y, const int32_t*
                                        out, static_cast<WsHeader*>(ws), shape->capacity > 0));
 }
 
+moe_status_t moe_selftest_wait_timeout(void* ws, uint32_t timeout_us, moe_stream_t stream) {
+  if (ws == nullptr || !aligned(ws, 16)) return MOE_ERR_WORKSPACE;
+  if (timeout_us < 1u || timeout_us > 2000000u) return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_wait_timeout_selftest(env_of(stream), static_cast<WsHeader*>(ws),
+                                                     uint64_t(timeout_us) * 1000u));
+}
+
 moe_status_t moe_get_device_error(void* ws, int32_t* detail, moe_stream_t stream) {
   if (ws == nullptr || !aligned(ws, 16)) return MOE_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -142,6 +142,10 @@ cudaError_t launch_dispatch_fp8(const LaunchEnv& env, const void* x, const int32
                                 int T, int H, int k, int64_t N, void* out, float* scales,
                                 WsHeader* hdr);
 
+// Self-test of the bounded-wait error path: a wait that nothing completes.
+cudaError_t launch_wait_timeout_selftest(const LaunchEnv& env, WsHeader* hdr,
+                                         uint64_t timeout_ns);
+
 // Round-robin router (diagnostic): ids[t,j] = (t*k + j) mod E, gates 1/k.
 cudaError_t launch_route_round_robin(const LaunchEnv& env, int T, int E, int k, int32_t* ids,
                                      float* gates);

@@ -319,6 +319,15 @@ moe_status_t moe_layout_noalloc(const moe_shape_t* shape, const int32_t* ids, in
                                 int32_t* expert_off, int32_t* rank_off, int32_t* rank_counts,
                                 int32_t* dst_pos, int32_t* src_idx, moe_stream_t stream);
 
+/* Self-test of the failure path of the kernels' bounded waits (the pages
+ * have no counterpart): launches one warp that waits on an mbarrier no copy
+ * will ever complete, with the same bounded wait the bulk-copy kernels use,
+ * for timeout_us microseconds (1 .. 2000000).  When it gives up it records
+ * MOE_ERR_DEVICE_TIMEOUT in the workspace header (detail = microseconds
+ * waited) and returns; nothing stays in flight and the context stays usable.
+ * Read the result with moe_get_device_error. */
+moe_status_t moe_selftest_wait_timeout(void* ws, uint32_t timeout_us, moe_stream_t stream);
+
 /* Synchronise `stream`, return the first device-side error recorded in `ws`
  * since the last read (MOE_OK if none) and clear it.  *detail (may be NULL)
  * receives the offending index (expert id, row, or block) when known. */
