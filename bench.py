@@ -576,7 +576,28 @@ def main():
         del g_op
         iso[name] = sorted(times)[len(times) // 2]
     iso_n = K_ops
-    del iso_buf
+
+    # the achievable floor for the same bytes: a plain device-to-device copy
+    # moving as many bytes (read + write) as dispatch and combine together,
+    # timed the same way (flushed L2, median)
+    _ab = algorithmic_bytes(w, kept_rows)
+    copy_bytes = (_ab["dispatch"] + _ab["combine"]) // 2 // 16 * 16
+    csrc = torch.empty(copy_bytes, dtype=torch.uint8, device=dev)
+    cdst = torch.empty_like(csrc)
+    csrc.fill_(3)
+    ctimes = []
+    for i in range(K_ops):
+        iso_buf.fill_(1)
+        iso_buf.view(torch.int64).sum()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        cdst.copy_(csrc)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ctimes.append(a.elapsed_time(b))
+    copy_ms = sorted(ctimes)[len(ctimes) // 2]
+    del csrc, cdst, iso_buf
 
     # end to end through the public API: every step copies its inputs in from
     # pinned host memory and its result back out.  Pipelined the way a server
@@ -694,6 +715,12 @@ def main():
                              "method": (f"in the step: a replay of the step with event records "
                                         f"between its kernels (no launch overlap across them), "
                                         f"mean of {K_ops}")},
+        "copy_anchor": {
+            "bytes_moved": 2 * copy_bytes, "us": round(copy_ms * 1e3, 2),
+            "gbs": round(2 * copy_bytes / (copy_ms * 1e-3) / 1e9, 1),
+            "dispatch_combine_over_copy": round((iso["dispatch"] + iso["combine"]) / copy_ms, 3),
+            "method": ("torch device-to-device copy of the same bytes as dispatch + combine "
+                       "(half read, half written), flushed L2, median")},
         "dispatch_combine_isolated": {
             "tokens_per_s": world * T / ((iso["dispatch"] + iso["combine"]) * 1e-3),
             "us": round((iso["dispatch"] + iso["combine"]) * 1e3, 2),
