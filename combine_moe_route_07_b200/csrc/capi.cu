@@ -279,6 +279,11 @@ moe_status_t moe_route_layout(const moe_shape_t* shape, const float* logits, con
   uint32_t* tables = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + kHeaderBytes);
   const size_t half = half_words_of(ws_bytes);
   const moe::LaunchEnv env = env_of(stream);
+  if (moe::route_layout_small_fits(shape->tokens, shape->experts, shape->k))
+    return from_cuda(moe::launch_route_layout_small(
+        env, logits, bias, shape->tokens, shape->experts, shape->k, shape->ranks,
+        (shape->flags & MOE_F_RENORM) ? 1 : 0, shape->capacity, shape->align, N, hdr, ids, gates,
+        counts, expert_off, rank_off, rank_counts, dst_pos, src_idx));
   if (shape->tokens > 0) {
     const cudaError_t err = moe::launch_route(env, logits, bias, shape->tokens, shape->experts,
                                               shape->k, (shape->flags & MOE_F_RENORM) ? 1 : 0,

@@ -146,6 +146,19 @@ cudaError_t launch_dispatch_fp8(const LaunchEnv& env, const void* x, const int32
 cudaError_t launch_wait_timeout_selftest(const LaunchEnv& env, WsHeader* hdr,
                                          uint64_t timeout_ns);
 
+// Steps 1-3 for a small batch in one launch of one thread-block cluster
+// (decode-sized): at most kSmallMaxAssign assignments and kSmallMaxExperts
+// experts.  Same results as launch_route + launch_layout.
+constexpr int kSmallMaxAssign = 4096;
+constexpr int kSmallMaxExperts = 512;
+bool route_layout_small_fits(int T, int E, int k);
+cudaError_t launch_route_layout_small(const LaunchEnv& env, const float* logits,
+                                      const float* bias, int T, int E, int k, int R, int renorm,
+                                      int capacity, int align, int64_t N, WsHeader* hdr,
+                                      int32_t* ids, float* gates, int32_t* counts,
+                                      int32_t* expert_off, int32_t* rank_off,
+                                      int32_t* rank_counts, int32_t* dst_pos, int32_t* src_idx);
+
 // Round-robin router (diagnostic): ids[t,j] = (t*k + j) mod E, gates 1/k.
 cudaError_t launch_route_round_robin(const LaunchEnv& env, int T, int E, int k, int32_t* ids,
                                      float* gates);
