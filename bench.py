@@ -603,62 +603,79 @@ def main():
     # pinned host memory and its result back out.  Pipelined the way a server
     # would run it: two device buffer sets, the next step's upload and the
     # previous step's download on their own streams, overlapping this step's
-    # kernels (which stay strictly one step at a time on the compute stream).
+    # kernels (which stay strictly one step at a time).  64 such steps are
+    # captured as one CUDA graph (copies, event edges and kernels) and
+    # replayed, so host launch overhead does not stand in for the copies.
     e2e = None
     if args.e2e_steps > 0:
         x_h = inp.x.pin_memory()
         lg_h = inp.logits.pin_memory()
         out_h = [torch.empty((T, w.H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-        set_a = (x, logits, out, g_step)
-        x, logits, out = torch.empty_like(x), torch.empty_like(logits), torch.empty_like(out)
+        set_a = (x, logits, out)
+        set_b = (torch.empty_like(x), torch.empty_like(logits), torch.empty_like(out))
+        sets = (set_a, set_b)
+
+        U = 64
+        cin, cout = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        x, logits, out = set_b
         shared = x if w.shared else None
         residual = x if w.residual else None
         step()  # the second set's first pass, outside capture
         torch.cuda.synchronize()
-        g_step_b = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_step_b):
-            step()
-        sets = (set_a, (x, logits, out, g_step_b))
-        x, logits, out, _ = set_a
+        g_e2e = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_e2e):
+            cap = torch.cuda.current_stream()
+            evs = []
+            for u in range(U):
+                bset = u % 2
+                xs, ls, os_ = sets[bset]
+                h2d_e, done_e, d2h_e = torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()
+                with torch.cuda.stream(cin):
+                    if u >= 2:
+                        cin.wait_event(evs[u - 2][1])  # step u-2 has finished reading this set
+                    else:
+                        cin.wait_stream(cap)
+                    xs.copy_(x_h, non_blocking=True)
+                    ls.copy_(lg_h, non_blocking=True)
+                    h2d_e.record(cin)
+                cap.wait_event(h2d_e)
+                if u >= 2:
+                    cap.wait_event(evs[u - 2][2])  # step u-2's result has left this set
+                x, logits, out = xs, ls, os_
+                shared = x if w.shared else None
+                residual = x if w.residual else None
+                step()
+                done_e.record(cap)
+                with torch.cuda.stream(cout):
+                    cout.wait_event(done_e)
+                    out_h[bset].copy_(os_, non_blocking=True)
+                    d2h_e.record(cout)
+                evs.append((h2d_e, done_e, d2h_e))
+            cap.wait_stream(cin)
+            cap.wait_stream(cout)
+        x, logits, out = set_a
         shared = x if w.shared else None
         residual = x if w.residual else None
-        cin, cout = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        h2d = [torch.cuda.Event() for _ in range(2)]
-        done = [torch.cuda.Event() for _ in range(2)]
-        d2h = [torch.cuda.Event() for _ in range(2)]
+        reps = max(1, -(-args.e2e_steps // U))
+        for _ in range(2):
+            g_e2e.replay()
+        torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        warm = 3
-        for it in range(warm + args.e2e_steps):
-            if it == warm:
-                torch.cuda.synchronize()
-                e0.record(stream)
-                cin.wait_event(e0)
-            bset = it % 2
-            xs, ls, os_, gs = sets[bset]
-            with torch.cuda.stream(cin):
-                cin.wait_event(done[bset])  # step it-2 has finished reading this set
-                xs.copy_(x_h, non_blocking=True)
-                ls.copy_(lg_h, non_blocking=True)
-                h2d[bset].record(cin)
-            stream.wait_event(h2d[bset])
-            stream.wait_event(d2h[bset])  # step it-2's result has left this set
-            gs.replay()
-            done[bset].record(stream)
-            with torch.cuda.stream(cout):
-                cout.wait_event(done[bset])
-                out_h[bset].copy_(os_, non_blocking=True)
-                d2h[bset].record(cout)
-        stream.wait_stream(cout)
+        e0.record(stream)
+        for _ in range(reps):
+            g_e2e.replay()
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dist, dev)
-        del g_step_b
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / (reps * U), dist, dev)
+        del g_e2e
         e2e = {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": x_h.numel() * 2 + lg_h.numel() * 4,
                "d2h_bytes_per_step": out_h[0].numel() * 2, "ms_per_step": e2e_ms,
+               "steps": reps * U,
                "mode": ("pipelined over two buffer sets: step i's kernels overlap step i+1's "
-                        "upload and step i-1's download (pinned host memory, own streams)")}
+                        "upload and step i-1's download (pinned host memory, own streams); "
+                        "64 steps per captured CUDA graph")}
 
     if rank != 0:
         if dist is not None:
