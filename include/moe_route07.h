@@ -19,13 +19,24 @@
  *   "Mixture-of-experts acceleration through overlap" (thecoregrid): the
  *      remote-owner-aligned layout (every row band bound to one destination).
  *
+ * Besides the four steps (moe_route, moe_layout, moe_dispatch, moe_combine,
+ * and the fused moe_route_layout / moe_route_layout_dispatch): the
+ * per-source-rank layout of a ragged exchange (moe_layout_src), rank-limited
+ * routing (moe_route_limited), the aux-loss-free bias update
+ * (moe_bias_update), the remote-first tile-aligned layout
+ * (moe_layout_remote_first), the round-robin router diagnostic
+ * (moe_route_round_robin), an allocation-free layout (moe_layout_noalloc) and
+ * a self-test of the kernels' failure path (moe_selftest_wait_timeout).
+ *
  * Everything runs on one GPU.  The R "ranks" are logical partitions of the
  * dispatched buffer: expert e belongs to rank e / (E/R), and each rank's rows
  * form one contiguous slice.
  *
  * Conventions for every call:
  *  - All pointers except `shape` are DEVICE pointers owned by the caller; the
- *    library allocates nothing and keeps no state between calls.
+ *    library allocates nothing and keeps no state between calls (beyond
+ *    host-side caches of launch parameters, and the static array of
+ *    moe_layout_noalloc).
  *  - Calls are asynchronous on `stream` (NULL = legacy default stream).  Only
  *    moe_get_device_error synchronises.
  *  - Arguments are checked on the host first; on MOE_ERR_INVALID_ARG nothing
