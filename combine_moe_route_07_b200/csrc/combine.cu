@@ -373,14 +373,15 @@ cudaError_t launch_combine(const LaunchEnv& env, const void* y, const int32_t* d
   }
   // Capacity mode drops most slots of a skewed batch: then each task moves
   // little and its latency dominates, so wider slices with the next task's
-  // metadata prefetched win; dense layouts do better with more warps.
+  // metadata prefetched win; dense layouts do better with more warps, all k
+  // slots' loads in flight at once.
   if (sparse && C8 >= 128) {
-    auto kern = combine_kernel<4, 2, 2, true>;
+    auto kern = combine_kernel<4, 2, 4, true>;
     const int grid = grid_for(kern, env, (int64_t)T * ((C8 + 127) / 128));
     return launch_pdl(env, kern, dim3(grid), dim3(kThreads), 0, ys, dst_pos, gates, sh, rs, T, H,
                       k, N, o, hdr);
   }
-  auto kern = combine_kernel<1, 4, 4, false>;
+  auto kern = combine_kernel<1, 8, 4, false>;
   const int grid = grid_for(kern, env, (int64_t)T * ((C8 + 31) / 32));
   return launch_pdl(env, kern, dim3(grid), dim3(kThreads), 0, ys, dst_pos, gates, sh, rs, T, H, k,
                     N, o, hdr);

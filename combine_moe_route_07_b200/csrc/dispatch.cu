@@ -378,7 +378,9 @@ cudaError_t launch_dispatch_bf16(const LaunchEnv& env, const void* x, const int3
   const char* xs = static_cast<const char*>(x);
   char* o = static_cast<char*>(out);
   const uint32_t row = (uint32_t)H * 2u;
-  if (row >= 1024 && row <= 32768) {
+  // The bulk pipeline pays off once each warp has several rows to stream;
+  // up to ~1k tokens one load and k stores per lane and slice finish sooner.
+  if (row >= 1024 && row <= 32768 && T >= 2048) {
     const int64_t warps = (int64_t)env.num_sms * kBulkWarps;  // one CTA per SM
     // slices of >= 1 KiB (16-byte multiples) when the tokens alone cannot
     // give every pipeline two units

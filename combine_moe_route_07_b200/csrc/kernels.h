@@ -148,8 +148,10 @@ cudaError_t launch_wait_timeout_selftest(const LaunchEnv& env, WsHeader* hdr,
 
 // Steps 1-3 for a small batch in one launch of one thread-block cluster
 // (decode-sized): at most kSmallMaxAssign assignments and kSmallMaxExperts
-// experts.  Same results as launch_route + launch_layout.
-constexpr int kSmallMaxAssign = 4096;
+// experts.  Same results as launch_route + launch_layout.  The cluster routes
+// on 8 SMs, one warp per token: at 128 tokens x 8 it saves a launch over the
+// two kernels; by 256 x 8 the two kernels' wider route has caught up.
+constexpr int kSmallMaxAssign = 1024;
 constexpr int kSmallMaxExperts = 512;
 bool route_layout_small_fits(int T, int E, int k);
 cudaError_t launch_route_layout_small(const LaunchEnv& env, const float* logits,
