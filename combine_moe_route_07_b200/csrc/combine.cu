@@ -77,9 +77,11 @@ __device__ __forceinline__ void fma8_x2(float (&acc)[8], float g, const uint4& v
 
 // One warp per (token, slice of 32*CPT chunks); lane j < k fetches the row
 // and gate of slot j once and the warp broadcasts them by shuffle.  With
-// PF the next task's rows and gates are fetched while this one computes, and
-// a batch of slots that are all dropped issues no loads at all (capacity mode
-// drops most slots of a skewed batch).
+// PF the next task's token, rows and gates are fetched while this one
+// computes.  KB == 1 walks only the kept slots (capacity mode drops most
+// slots of a skewed batch), a token with no kept slot and no shared or
+// residual row just stores zeros; KB > 1 keeps KB slots' loads in flight
+// and skips a batch whose slots are all dropped.
 template <int CPT, int KB, int MINB, bool PF>
 __global__ void __launch_bounds__(kThreads, MINB)
     combine_kernel(const char* __restrict__ y, const int32_t* __restrict__ dst_pos,
@@ -94,12 +96,13 @@ __global__ void __launch_bounds__(kThreads, MINB)
   const int64_t tasks = (int64_t)T * S;
   const size_t row_bytes = (size_t)H * 2;
   const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
-  // slot j of task `task` (lane j < k), -1 when dropped or out of range
-  auto fetch = [&](int64_t task, int& p, float& g) {
+  // token of task `task` and slot j of it (lane j < k), -1 when dropped or
+  // out of range
+  auto fetch = [&](int64_t task, int& t, int& p, float& g) {
+    t = task < tasks ? (int)((uint32_t)task / (uint32_t)S) : 0;  // tasks < 2^31 (host check)
     p = -1;
     g = 0.0f;
     if (task < tasks && lane < k) {
-      const int t = (int)((uint32_t)task / (uint32_t)S);  // tasks < 2^31 (host check)
       p = __ldg(dst_pos + (size_t)t * k + lane);
       g = __ldg(gates + (size_t)t * k + lane);
       if (p >= N) {
@@ -109,68 +112,94 @@ __global__ void __launch_bounds__(kThreads, MINB)
     }
   };
   int64_t task = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
-  int pl, pn = -1;
+  int tl, pl, tn = 0, pn = -1;
   float gl, gn = 0.0f;
-  fetch(task, pl, gl);
+  fetch(task, tl, pl, gl);
   for (; task < tasks; task += nw) {
-    if (PF) fetch(task + nw, pn, gn);
-    const int t = (int)((uint32_t)task / (uint32_t)S);
+    if (PF) fetch(task + nw, tn, pn, gn);
+    const int t = PF ? tl : (int)((uint32_t)task / (uint32_t)S);
     const int cb = (int)((uint32_t)task - (uint32_t)t * (uint32_t)S) * 32 * CPT + lane;
     const unsigned kept = __ballot_sync(kFull, pl >= 0);
-    float acc[CPT][8];
+    if (KB == 1 && kept == 0u && shared == nullptr && residual == nullptr) {
 #pragma unroll
-    for (int i = 0; i < CPT; ++i)
+      for (int i = 0; i < CPT; ++i) {
+        const int c = cb + 32 * i;
+        if (c < C8) st16(out + (size_t)t * row_bytes + (size_t)c * 16, make_uint4(0, 0, 0, 0));
+      }
+    } else {
+      float acc[CPT][8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[i][e] = 0.0f;
+      for (int i = 0; i < CPT; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[i][e] = 0.0f;
 
-    for (int j0 = 0; j0 < k; j0 += KB) {
-      if (((kept >> j0) & ((1u << KB) - 1u)) == 0u) continue;  // every slot dropped
-      uint4 v[KB][CPT];
-      float gw[KB];
-      int pp[KB];
+      if constexpr (KB == 1) {
+        for (unsigned m = kept; m != 0u; m &= m - 1u) {  // kept slots, ascending
+          const int j = __ffs(m) - 1;
+          const int p = __shfl_sync(kFull, pl, j);
+          const float g = __shfl_sync(kFull, gl, j);
+          const char* src = y + (size_t)p * row_bytes;
+          uint4 v[CPT];
 #pragma unroll
-      for (int jj = 0; jj < KB; ++jj) {
-        const int j = j0 + jj;  // j < 32: the shuffle source is always a lane
-        pp[jj] = __shfl_sync(kFull, pl, j & 31);
-        gw[jj] = __shfl_sync(kFull, gl, j & 31);
-        if (j >= k) pp[jj] = -1;
-        const char* src = y + (size_t)(pp[jj] < 0 ? 0 : pp[jj]) * row_bytes;
+          for (int i = 0; i < CPT; ++i) {
+            const int c = cb + 32 * i;
+            v[i] = c < C8 ? ld16_stream(src + (size_t)c * 16) : make_uint4(0, 0, 0, 0);
+          }
 #pragma unroll
-        for (int i = 0; i < CPT; ++i) {
-          const int c = cb + 32 * i;
-          if (pp[jj] >= 0 && c < C8)
-            v[jj][i] = ld16_stream(src + (size_t)c * 16);
-          else
-            v[jj][i] = make_uint4(0, 0, 0, 0);
+          for (int i = 0; i < CPT; ++i) fma8(acc[i], g, v[i]);
+        }
+      } else {
+        for (int j0 = 0; j0 < k; j0 += KB) {
+          if (((kept >> j0) & ((1u << KB) - 1u)) == 0u) continue;  // every slot dropped
+          uint4 v[KB][CPT];
+          float gw[KB];
+          int pp[KB];
+#pragma unroll
+          for (int jj = 0; jj < KB; ++jj) {
+            const int j = j0 + jj;  // j < 32: the shuffle source is always a lane
+            pp[jj] = __shfl_sync(kFull, pl, j & 31);
+            gw[jj] = __shfl_sync(kFull, gl, j & 31);
+            if (j >= k) pp[jj] = -1;
+            const char* src = y + (size_t)(pp[jj] < 0 ? 0 : pp[jj]) * row_bytes;
+#pragma unroll
+            for (int i = 0; i < CPT; ++i) {
+              const int c = cb + 32 * i;
+              if (pp[jj] >= 0 && c < C8)
+                v[jj][i] = ld16_stream(src + (size_t)c * 16);
+              else
+                v[jj][i] = make_uint4(0, 0, 0, 0);
+            }
+          }
+#pragma unroll
+          for (int jj = 0; jj < KB; ++jj)
+            if (pp[jj] >= 0) {
+#pragma unroll
+              for (int i = 0; i < CPT; ++i) fma8(acc[i], gw[jj], v[jj][i]);
+            }
         }
       }
-#pragma unroll
-      for (int jj = 0; jj < KB; ++jj)
-        if (pp[jj] >= 0) {
-#pragma unroll
-          for (int i = 0; i < CPT; ++i) fma8(acc[i], gw[jj], v[jj][i]);
-        }
-    }
 
 #pragma unroll
-    for (int i = 0; i < CPT; ++i) {
-      const int c = cb + 32 * i;
-      if (c >= C8) continue;
-      const size_t off = (size_t)t * row_bytes + (size_t)c * 16;
-      if (shared != nullptr) add8(acc[i], ld16_stream(shared + off));
-      if (residual != nullptr) add8(acc[i], ld16_stream(residual + off));
-      uint4 o;
-      o.x = pack_bf16x2(acc[i][0], acc[i][1]);
-      o.y = pack_bf16x2(acc[i][2], acc[i][3]);
-      o.z = pack_bf16x2(acc[i][4], acc[i][5]);
-      o.w = pack_bf16x2(acc[i][6], acc[i][7]);
-      st16(out + off, o);
+      for (int i = 0; i < CPT; ++i) {
+        const int c = cb + 32 * i;
+        if (c >= C8) continue;
+        const size_t off = (size_t)t * row_bytes + (size_t)c * 16;
+        if (shared != nullptr) add8(acc[i], ld16_stream(shared + off));
+        if (residual != nullptr) add8(acc[i], ld16_stream(residual + off));
+        uint4 o;
+        o.x = pack_bf16x2(acc[i][0], acc[i][1]);
+        o.y = pack_bf16x2(acc[i][2], acc[i][3]);
+        o.z = pack_bf16x2(acc[i][4], acc[i][5]);
+        o.w = pack_bf16x2(acc[i][6], acc[i][7]);
+        st16(out + off, o);
+      }
     }
     if (PF) {
+      tl = tn;
       pl = pn;
       gl = gn;
     } else {
-      fetch(task + nw, pl, gl);
+      fetch(task + nw, tl, pl, gl);
     }
   }
 }
@@ -373,10 +402,11 @@ cudaError_t launch_combine(const LaunchEnv& env, const void* y, const int32_t* d
   }
   // Capacity mode drops most slots of a skewed batch: then each task moves
   // little and its latency dominates, so wider slices with the next task's
-  // metadata prefetched win; dense layouts do better with more warps, all k
-  // slots' loads in flight at once.
+  // metadata prefetched win, one slot at a time (a slot's loads are skipped
+  // alone when it is dropped, and nothing spills at 64 registers); dense
+  // layouts do better with more warps, all k slots' loads in flight at once.
   if (sparse && C8 >= 128) {
-    auto kern = combine_kernel<4, 2, 4, true>;
+    auto kern = combine_kernel<4, 1, 4, true>;
     const int grid = grid_for(kern, env, (int64_t)T * ((C8 + 127) / 128));
     return launch_pdl(env, kern, dim3(grid), dim3(kThreads), 0, ys, dst_pos, gates, sh, rs, T, H,
                       k, N, o, hdr);
