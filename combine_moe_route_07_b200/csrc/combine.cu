@@ -204,7 +204,8 @@ __global__ void __launch_bounds__(kThreads, MINB)
   }
 }
 
-// Bulk variant.  One CTA of kBulkWarps warps per SM; warp w owns a contiguous
+// Bulk variant.  One CTA per SM of 24 warps (16 when the stages of k plus the
+// shared and residual slots do not fit twice per warp for 24); warp w owns a contiguous
 // range of units (token t, 512-byte slice s of the row), so consecutive units
 // mostly share a token and its dst_pos/gates (fetched one token ahead).  Per
 // warp, a ring of `ns` shared-memory stages each holds one unit: the kept
@@ -215,22 +216,23 @@ __global__ void __launch_bounds__(kThreads, MINB)
 // slice.  Waits are bounded: a stage that does not fill within a second sets
 // MOE_ERR_DEVICE_TIMEOUT, and the warp waits (bounded) for its copies still in
 // flight before it exits.
-constexpr int kBulkWarps = 16;
+constexpr int kBulkMaxWarps = 24;
+constexpr int kBulkMinWarps = 16;
 constexpr int kBulkMaxStages = 8;
 constexpr uint32_t kBulkSlice = 512;
 constexpr size_t kBulkSmemBudget = 200u * 1024u;
 constexpr uint64_t kBulkTimeoutNs = 1000000000ull;
 
 template <int KMAX>
-__global__ void __launch_bounds__(kBulkWarps * 32, 1)
+__global__ void __launch_bounds__(kBulkMaxWarps * 32, 1)
     combine_bulk_kernel(const char* __restrict__ y, const int32_t* __restrict__ dst_pos,
                         const float* __restrict__ gates, const char* __restrict__ shared,
                         const char* __restrict__ residual, int T, int H, int k, int64_t N,
                         char* __restrict__ out, WsHeader* hdr, int ns, uint32_t stage_bytes) {
   extern __shared__ __align__(128) unsigned char sbuf[];
-  __shared__ uint64_t bars[kBulkWarps][kBulkMaxStages];
-  __shared__ float sgate[kBulkWarps][kBulkMaxStages][32];  // gate of each slot, per stage
-  __shared__ uint32_t skept[kBulkWarps][kBulkMaxStages];   // kept-slot mask, per stage
+  __shared__ uint64_t bars[kBulkMaxWarps][kBulkMaxStages];
+  __shared__ float sgate[kBulkMaxWarps][kBulkMaxStages][32];  // gate of each slot, per stage
+  __shared__ uint32_t skept[kBulkMaxWarps][kBulkMaxStages];   // kept-slot mask, per stage
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t row = (uint32_t)H * 2;
   const int nsl = (int)((row + kBulkSlice - 1) / kBulkSlice);
@@ -245,8 +247,8 @@ __global__ void __launch_bounds__(kBulkWarps * 32, 1)
   pdl_wait();  // y, gates and dst_pos may come from the kernel launched just before
   pdl_trigger();
   const int64_t units = (int64_t)T * nsl;
-  const int64_t nwarps = (int64_t)gridDim.x * kBulkWarps;
-  const int64_t wid = (int64_t)blockIdx.x * kBulkWarps + w;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + w;
   const int64_t u0 = units * wid / nwarps, u1 = units * (wid + 1) / nwarps;
   if (u0 >= u1) return;
   const int nunits = (int)(u1 - u0);
@@ -383,22 +385,25 @@ cudaError_t launch_combine(const LaunchEnv& env, const void* y, const int32_t* d
   char* o = static_cast<char*>(out);
   // Dense layouts with at least 8 row slices per warp of a full bulk grid:
   // the bulk variant, when the stages of up to 12 slots (k plus the shared
-  // and residual rows) fit twice per warp.
+  // and residual rows) fit twice per warp.  More warps beat deeper rings:
+  // 24 warps with two stages each run the Prefill combine 2 µs faster than
+  // 16 with three; wider slices with fewer warps ran far slower.
   const int extra = (shared != nullptr) + (residual != nullptr);
   const uint32_t stage_bytes = (uint32_t)(k + extra) * kBulkSlice;
-  const int ns_fit = (int)(kBulkSmemBudget / ((size_t)kBulkWarps * stage_bytes));
+  const int W = kBulkSmemBudget / ((size_t)kBulkMaxWarps * stage_bytes) >= 2 ? kBulkMaxWarps
+                                                                             : kBulkMinWarps;
+  const int ns_fit = (int)(kBulkSmemBudget / ((size_t)W * stage_bytes));
   const int64_t slices = (int64_t)T * ((2 * (int64_t)H + kBulkSlice - 1) / kBulkSlice);
-  if (!sparse && k <= 16 && ns_fit >= 2 &&
-      slices >= 8 * (int64_t)env.num_sms * kBulkWarps) {
+  if (!sparse && k <= 16 && ns_fit >= 2 && slices >= 8 * (int64_t)env.num_sms * W) {
     const int ns = ns_fit < kBulkMaxStages ? ns_fit : kBulkMaxStages;
-    const size_t smem = (size_t)kBulkWarps * ns * stage_bytes;
+    const size_t smem = (size_t)W * ns * stage_bytes;
     auto kern = k <= 8 ? combine_bulk_kernel<8> : combine_bulk_kernel<16>;
     int per_sm = 1;
     const cudaError_t err =
-        blocks_per_sm(reinterpret_cast<const void*>(kern), kBulkWarps * 32, smem, &per_sm);
+        blocks_per_sm(reinterpret_cast<const void*>(kern), W * 32, smem, &per_sm);
     if (err != cudaSuccess) return err;
-    return launch_pdl(env, kern, dim3((unsigned)(env.num_sms * per_sm)), dim3(kBulkWarps * 32),
-                      smem, ys, dst_pos, gates, sh, rs, T, H, k, N, o, hdr, ns, stage_bytes);
+    return launch_pdl(env, kern, dim3((unsigned)(env.num_sms * per_sm)), dim3(W * 32), smem, ys,
+                      dst_pos, gates, sh, rs, T, H, k, N, o, hdr, ns, stage_bytes);
   }
   // Capacity mode drops most slots of a skewed batch: then each task moves
   // little and its latency dominates, so wider slices with the next task's
