@@ -36,7 +36,7 @@ __global__ void __launch_bounds__(kThreads)
   // dynamic: [hist: E int32, padded to 16 B] (HIST), [rows: kWarps x 2 x E floats] (STAGE),
   // [rank limit: kWarps x (R + ceil(R/32)) words] (M < R), [bias: E floats] (STAGE)
   extern __shared__ __align__(16) unsigned char dyn[];
-  __shared__ uint32_t cand_all[kWarps][NK >= 8 ? 3 * kMaxCand : 1];
+  __shared__ __align__(16) uint32_t cand_all[kWarps][NK >= 8 ? 3 * kMaxCand : 1];
   __shared__ uint64_t bars[kWarps][2];
   int32_t* hist = reinterpret_cast<int32_t*>(dyn);
   const size_t hist_bytes = HIST ? (((size_t)E * 4 + 15) & ~(size_t)15) : 0;

@@ -10,8 +10,8 @@
 // is two hardware warp reductions (redux.sync): the largest code, then the
 // lowest expert id among the lanes holding it, which is the tie rule.  Three
 // forms of the same selection: route_tokens (every code, k rounds; E <= 224),
-// route_token_thr (a threshold first, then the rounds over the few keys
-// above it) and route_token_smem (the threshold form with the row and the
+// route_token_thr (a threshold first, then the few keys above it ranked
+// against each other) and route_token_smem (the threshold form with the row and the
 // bias read from shared memory, only the codes in registers).  An optional
 // rank limit clears the codes of all but the M best ranks first.  The gates
 // are a softmax of the selected RAW logits evaluated in fp64 (k values per
@@ -305,12 +305,59 @@ __device__ __forceinline__ int route_tokens(const float* __restrict__ logits, co
 // Exact top-k through a threshold, for many keys per lane (NK >= 8).
 // tau = the k-th largest of the 32 lane maxima: those k maxima are k distinct
 // keys >= tau, so the k-th largest key is >= tau and no key below tau can be
-// selected.  The warp compacts the keys >= tau (usually k to 2k of them) into
-// shared memory and runs the k selection rounds over at most two per lane.
-// More than kMaxCand candidates (heavy ties) falls back to route_tokens.
-// `cand` is this warp's 3*kMaxCand words of shared memory.  (Rows staged in
-// shared memory go through route_token_smem instead.)
+// selected.  The warp compacts the keys >= tau (usually k to k+4 of them) into
+// shared memory and ranks them (select_ranked).  More than kMaxCand candidates
+// (heavy ties) falls back to route_tokens.  `cand` is this warp's 3*kMaxCand
+// words of shared memory, 8-byte aligned.  (Rows staged in shared memory go
+// through route_token_smem instead.)
 constexpr int kMaxCand = 64;
+
+// Slot order of `total` candidates: the key (code << 32) | ~id orders larger
+// codes first and, among equal codes, lower ids first, and no two keys are
+// equal, so candidate i's slot is the number of keys above its own.  Lanes i
+// and i+32 rank candidates i and i+32 against every key (one broadcast load
+// each), the candidates of slots j < k are scattered to slot j, and lane j < k
+// returns slot j's expert (and, with RAW, its raw logit bits from `raw`).
+// `key` holds kMaxCand keys and `raw` kMaxCand words; both are reused for the
+// slots, and the warp is synchronised before they are written and on return.
+template <bool RAW>
+__device__ __forceinline__ void select_ranked(uint64_t* key, uint32_t* raw, int total, int k,
+                                              int lane, int& sel_e, uint32_t& sel_raw) {
+  const bool h0 = lane < total, h1 = lane + 32 < total;
+  const uint64_t k0 = h0 ? key[lane] : 0ull;
+  const uint64_t k1 = h1 ? key[lane + 32] : 0ull;
+  uint32_t v0 = 0u, v1 = 0u;
+  if (RAW) {
+    v0 = h0 ? raw[lane] : 0u;
+    v1 = h1 ? raw[lane + 32] : 0u;
+  }
+  int n0 = 0, n1 = 0;
+  if (total <= 32) {
+    for (int m = 0; m < total; ++m) n0 += key[m] > k0 ? 1 : 0;
+  } else {
+    for (int m = 0; m < total; ++m) {
+      const uint64_t km = key[m];
+      n0 += km > k0 ? 1 : 0;
+      n1 += km > k1 ? 1 : 0;
+    }
+  }
+  __syncwarp();  // every key has been read: the slots reuse the arrays
+  uint32_t* slot_e = reinterpret_cast<uint32_t*>(key);
+  if (h0 && n0 < k) {
+    slot_e[n0] = ~(uint32_t)k0;
+    if (RAW) raw[n0] = v0;
+  }
+  if (h1 && n1 < k) {
+    slot_e[n1] = ~(uint32_t)k1;
+    if (RAW) raw[n1] = v1;
+  }
+  __syncwarp();
+  if (lane < k) {
+    sel_e = (int)slot_e[lane];
+    if (RAW) sel_raw = raw[lane];
+  }
+  __syncwarp();  // the next token may overwrite the arrays
+}
 
 template <int NK>
 __device__ __forceinline__ int route_token_thr(const float* __restrict__ logits, int t, int T,
@@ -367,55 +414,20 @@ __device__ __forceinline__ int route_token_thr(const float* __restrict__ logits,
     if (lane >= o) pre += y;
   }
   pre -= c;
+  uint64_t* ckey = reinterpret_cast<uint64_t*>(cand);
+  uint32_t* craw = cand + 2 * kMaxCand;
 #pragma unroll
   for (int i = 0; i < NK; ++i)
     if (code[i] != 0u && code[i] >= tau) {
-      cand[pre] = code[i];
-      cand[kMaxCand + pre] = (uint32_t)(lane + 32 * i);
-      cand[2 * kMaxCand + pre] = __float_as_uint(raw[i]);
+      ckey[pre] = ((uint64_t)code[i] << 32) | (uint64_t)(~(uint32_t)(lane + 32 * i));
+      craw[pre] = __float_as_uint(raw[i]);
       ++pre;
     }
   __syncwarp();
-  uint32_t c0 = 0u, c1 = 0u, e0 = 0u, e1 = 0u;
-  float r0 = 0.0f, r1 = 0.0f;
-  if (lane < total) {
-    c0 = cand[lane];
-    e0 = cand[kMaxCand + lane];
-    r0 = __uint_as_float(cand[2 * kMaxCand + lane]);
-  }
-  if (lane + 32 < total) {
-    c1 = cand[lane + 32];
-    e1 = cand[kMaxCand + lane + 32];
-    r1 = __uint_as_float(cand[2 * kMaxCand + lane + 32]);
-  }
-  __syncwarp();  // the next token may overwrite cand
-
-  float sel_raw = 0.0f;
   sel_e = 0;
-  for (int j = 0; j < k; ++j) {
-    const bool use1 = (c1 > c0) || (c1 == c0 && c1 != 0u && e1 < e0);
-    const uint32_t bk = use1 ? c1 : c0;
-    const uint32_t be = use1 ? e1 : e0;
-    const uint32_t top = __reduce_max_sync(kFull, bk);
-    const uint32_t win = __reduce_min_sync(kFull, (bk == top) ? be : 0xffffffffu);
-    const bool mine = (bk == top) && (be == win);
-    float r = 0.0f;
-    if (mine) {
-      if (use1) {
-        c1 = 0u;
-        r = r1;
-      } else {
-        c0 = 0u;
-        r = r0;
-      }
-    }
-    const unsigned holder = __ballot_sync(kFull, mine);
-    r = __shfl_sync(kFull, r, __ffs(holder) - 1);
-    if (lane == j) {
-      sel_e = (int)win;
-      sel_raw = r;
-    }
-  }
+  uint32_t rbits = 0u;
+  select_ranked<true>(ckey, craw, total, k, lane, sel_e, rbits);
+  const float sel_raw = __uint_as_float(rbits);
 
   if (renorm) {
     const float m = warp_max_f(lane < k ? sel_raw : -INFINITY);
@@ -578,41 +590,17 @@ __device__ __forceinline__ int route_token_smem(const float* srow, const float* 
       if (lane >= o) pre += y;
     }
     pre -= c;
+    uint64_t* ckey = reinterpret_cast<uint64_t*>(cand);
 #pragma unroll
     for (int i = 0; i < NK; ++i)
       if (code[i] != 0u && code[i] >= tau) {
-        cand[pre] = code[i];
-        cand[kMaxCand + pre] = (uint32_t)(lane + 32 * i);
+        ckey[pre] = ((uint64_t)code[i] << 32) | (uint64_t)(~(uint32_t)(lane + 32 * i));
         ++pre;
       }
     __syncwarp();
-    uint32_t c0 = 0u, c1 = 0u, e0 = 0u, e1 = 0u;
-    if (lane < total) {
-      c0 = cand[lane];
-      e0 = cand[kMaxCand + lane];
-    }
-    if (lane + 32 < total) {
-      c1 = cand[lane + 32];
-      e1 = cand[kMaxCand + lane + 32];
-    }
-    __syncwarp();  // the next token may overwrite cand
-    for (int j = 0; j < k; ++j) {
-      const bool use1 = (c1 > c0) || (c1 == c0 && c1 != 0u && e1 < e0);
-      const uint32_t bk = use1 ? c1 : c0;
-      const uint32_t be = use1 ? e1 : e0;
-      const uint32_t top = __reduce_max_sync(kFull, bk);
-      const uint32_t win = __reduce_min_sync(kFull, (bk == top) ? be : 0xffffffffu);
-      if (bk == top && be == win) {
-        if (use1)
-          c1 = 0u;
-        else
-          c0 = 0u;
-      }
-      if (lane == j) {
-        sel_e = (int)win;
-        sel_raw = srow[win];
-      }
-    }
+    uint32_t unused = 0u;
+    select_ranked<false>(ckey, cand + 2 * kMaxCand, total, k, lane, sel_e, unused);
+    if (lane < k) sel_raw = srow[sel_e];
   }
 
   if (renorm) {

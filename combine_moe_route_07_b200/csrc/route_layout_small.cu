@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) route_layout_small_kernel(co
   // kept[E], wh[kSmallWarps][E] per-warp counts then bases, sid[TB*k] ids,
   // srk[TB*k] ranks in the warp's run
   extern __shared__ int32_t sm[];
-  __shared__ uint32_t cand_all[kSmallWarps][NK >= 8 ? 3 * kMaxCand : 1];
+  __shared__ __align__(16) uint32_t cand_all[kSmallWarps][NK >= 8 ? 3 * kMaxCand : 1];
   __shared__ int32_t wtot[kSmallWarps];
   cg::cluster_group cluster = cg::this_cluster();
   const int T = P.T, E = P.E, k = P.k, C = P.capacity;
