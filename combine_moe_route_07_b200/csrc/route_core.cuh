@@ -15,7 +15,11 @@
 // bias read from shared memory, only the codes in registers).  An optional
 // rank limit clears the codes of all but the M best ranks first.  The gates
 // are a softmax of the selected RAW logits evaluated in fp64 (k values per
-// token) and rounded to fp32 once.
+// token): fp64 exponentials and sum, the quotient as the exponential times the
+// correctly rounded fp64 reciprocal of the sum (a full fp64 division cost ~80
+// more instructions per token), then one rounding to fp32.  That differs from
+// rounding the exact fp64 quotient only when it lies within ~2^-52 of an fp32
+// rounding boundary, far inside the 1e-6 gate tolerance.
 #pragma once
 
 #include <math.h>
@@ -284,7 +288,7 @@ __device__ __forceinline__ int route_tokens(const float* __restrict__ logits, co
       const float m = warp_max_f(lane < k ? sel_raw[u] : -INFINITY);
       const double ex = (lane < k) ? exp((double)sel_raw[u] - (double)m) : 0.0;
       const double den = warp_sum_d(ex);
-      gate[u] = (float)(ex / den);
+      gate[u] = (float)(ex * __drcp_rn(den));
     } else {
       float lm = -INFINITY;
 #pragma unroll
@@ -295,7 +299,7 @@ __device__ __forceinline__ int route_tokens(const float* __restrict__ logits, co
       for (int i = 0; i < NK; ++i)
         if (lane + 32 * i < E) part += exp((double)raw[u][i] - (double)m);
       const double den = warp_sum_d(part);
-      gate[u] = (float)(exp((double)sel_raw[u] - (double)m) / den);
+      gate[u] = (float)(exp((double)sel_raw[u] - (double)m) * __drcp_rn(den));
     }
   }
   return nan_tok;
@@ -433,7 +437,7 @@ __device__ __forceinline__ int route_token_thr(const float* __restrict__ logits,
     const float m = warp_max_f(lane < k ? sel_raw : -INFINITY);
     const double ex = (lane < k) ? exp((double)sel_raw - (double)m) : 0.0;
     const double den = warp_sum_d(ex);
-    gate = (float)(ex / den);
+    gate = (float)(ex * __drcp_rn(den));
   } else {
     float lm = -INFINITY;
 #pragma unroll
@@ -444,7 +448,7 @@ __device__ __forceinline__ int route_token_thr(const float* __restrict__ logits,
     for (int i = 0; i < NK; ++i)
       if (lane + 32 * i < E) part += exp((double)raw[i] - (double)m);
     const double den = warp_sum_d(part);
-    gate = (float)(exp((double)sel_raw - (double)m) / den);
+    gate = (float)(exp((double)sel_raw - (double)m) * __drcp_rn(den));
   }
   return nan_tok;
 }
@@ -607,7 +611,7 @@ __device__ __forceinline__ int route_token_smem(const float* srow, const float* 
     const float m = warp_max_f(lane < k ? sel_raw : -INFINITY);
     const double ex = (lane < k) ? exp((double)sel_raw - (double)m) : 0.0;
     const double den = warp_sum_d(ex);
-    gate = (float)(ex / den);
+    gate = (float)(ex * __drcp_rn(den));
   } else {
     float lm = -INFINITY;
 #pragma unroll
@@ -619,7 +623,7 @@ __device__ __forceinline__ int route_token_smem(const float* srow, const float* 
     for (int i = 0; i < NK; ++i)
       if (lane + 32 * i < E) part += exp((double)srow[lane + 32 * i] - (double)m);
     const double den = warp_sum_d(part);
-    gate = (float)(exp((double)sel_raw - (double)m) / den);
+    gate = (float)(exp((double)sel_raw - (double)m) * __drcp_rn(den));
   }
   return nan_tok;
 }

@@ -5,7 +5,8 @@ Tolerances (from the arithmetic, stated once here):
   ids, counts, offsets, dst_pos, src_idx, dispatched bf16 rows, e4m3 codes and
   fp32 scales: bit-exact (integer work, copies, and fp32 decisions taken in the
   same precision on both sides);
-  gates: 1e-6 relative (GPU fp64 softmax rounded once vs the oracle's fp64);
+  gates: 1e-6 relative (GPU fp64 softmax with a reciprocal-multiply, rounded to
+  fp32 once, vs the oracle's fp64 division: at most one fp32 ulp apart);
   combine: 1 bf16 ulp (GPU fp32 slot-order FMAs vs the oracle's fp64 sum, both
   rounded once to bf16; the fp32 error is far below half a bf16 ulp, so only
   values next to a rounding midpoint can land one ulp apart).
