@@ -558,9 +558,10 @@ __device__ __forceinline__ int route_token_smem(const float* srow, const float* 
     const unsigned hold = __ballot_sync(kFull, mm == top);
     if (lane == __ffs(hold) - 1) mm = 0u;
   }
-  int c = 0;
+  uint32_t cmask = 0u;  // bit i: key i of this lane is a candidate
 #pragma unroll
-  for (int i = 0; i < NK; ++i) c += (code[i] != 0u && code[i] >= tau) ? 1 : 0;
+  for (int i = 0; i < NK; ++i) cmask |= (code[i] != 0u && code[i] >= tau) ? (1u << i) : 0u;
+  const int c = __popc(cmask);
   const int total = (int)__reduce_add_sync(kFull, (unsigned)c);
 
   float sel_raw = 0.0f;
@@ -594,13 +595,15 @@ __device__ __forceinline__ int route_token_smem(const float* srow, const float* 
       if (lane >= o) pre += y;
     }
     pre -= c;
+    // only the few candidate keys are visited; their codes are formed again
+    // from the staged row (a candidate's rank is kept, so no mask applies)
     uint64_t* ckey = reinterpret_cast<uint64_t*>(cand);
-#pragma unroll
-    for (int i = 0; i < NK; ++i)
-      if (code[i] != 0u && code[i] >= tau) {
-        ckey[pre] = ((uint64_t)code[i] << 32) | (uint64_t)(~(uint32_t)(lane + 32 * i));
-        ++pre;
-      }
+    for (uint32_t m = cmask; m != 0u; m &= m - 1u) {
+      const int e = lane + 32 * (__ffs(m) - 1);
+      const uint32_t ce = order_code(__fadd_rn(srow[e], sbias[e]));
+      ckey[pre] = ((uint64_t)ce << 32) | (uint64_t)(~(uint32_t)e);
+      ++pre;
+    }
     __syncwarp();
     uint32_t unused = 0u;
     select_ranked<false>(ckey, cand + 2 * kMaxCand, total, k, lane, sel_e, unused);
