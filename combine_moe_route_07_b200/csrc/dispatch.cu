@@ -269,8 +269,12 @@ __global__ void __launch_bounds__(kThreads)
 // aligned lanes, its amax a 3-step xor shuffle), writes the codes and scales
 // into one of kFp8Stages shared-memory stages; lane 0 issues the k bulk
 // stores of the codes row (one bulk group per token) and the lanes write the
-// k copies of the scales row with ordinary coalesced stores.
+// k copies of the scales row with ordinary coalesced stores.  The first
+// kFp8PrefetchGroups groups of the warp's next token are loaded into
+// registers as soon as this token is quantised, so their latency hides
+// behind this token's stores and the wait for a free stage.
 constexpr int kFp8Stages = 4;
+constexpr int kFp8PrefetchGroups = 4;
 
 __global__ void __launch_bounds__(kBulkWarps * 32)
     dispatch_fp8_bulk_kernel(const char* __restrict__ x, const int32_t* __restrict__ dst_pos,
@@ -288,6 +292,21 @@ __global__ void __launch_bounds__(kBulkWarps * 32)
   const int64_t stride = (int64_t)gridDim.x * kBulkWarps;
   int64_t t = (int64_t)blockIdx.x * kBulkWarps + w;
   int pl = (t < T && lane < k) ? __ldg(dst_pos + (size_t)t * k + lane) : -1;
+  // the first groups of token tt, 32 bytes a lane each
+  const int pf = groups < kFp8PrefetchGroups ? groups : kFp8PrefetchGroups;
+  uint4 nx[2 * kFp8PrefetchGroups];
+  auto prefetch = [&](int64_t tt) {
+    const char* src = x + (size_t)tt * xrow;
+#pragma unroll
+    for (int g = 0; g < kFp8PrefetchGroups; ++g) {
+      const int ch = 512 * g + 16 * lane;
+      if (tt < T && g < pf) {
+        nx[2 * g] = ld16_stream(src + (size_t)ch * 2);
+        nx[2 * g + 1] = ld16_stream(src + (size_t)ch * 2 + 16);
+      }
+    }
+  };
+  prefetch(t);
   for (int64_t i = 0; t < T; ++i, t += stride) {
     const int s = (int)(i % kFp8Stages);
     unsigned char* sp = st + (size_t)s * stage_bytes;
@@ -297,11 +316,8 @@ __global__ void __launch_bounds__(kBulkWarps * 32)
     if (lane == 0) bulk_wait_read<kFp8Stages - 1>();
     __syncwarp();
     const char* src = x + (size_t)t * xrow;
-#pragma unroll 4
-    for (int g = 0; g < groups; ++g) {
+    auto quantise = [&](int g, const uint4& v0, const uint4& v1) {
       const int ch = 512 * g + 16 * lane;
-      const uint4 v0 = ld16_stream(src + (size_t)ch * 2);
-      const uint4 v1 = ld16_stream(src + (size_t)ch * 2 + 16);
       float f[16] = {bf16lo(v0.x), bf16hi(v0.x), bf16lo(v0.y), bf16hi(v0.y),
                      bf16lo(v0.z), bf16hi(v0.z), bf16lo(v0.w), bf16hi(v0.w),
                      bf16lo(v1.x), bf16hi(v1.x), bf16lo(v1.y), bf16hi(v1.y),
@@ -325,7 +341,16 @@ __global__ void __launch_bounds__(kBulkWarps * 32)
       }
       *reinterpret_cast<uint4*>(sp + ch) = q;
       if ((lane & 7) == 0) *reinterpret_cast<float*>(sp + H + 4 * (ch >> 7)) = scale;
+    };
+#pragma unroll
+    for (int g = 0; g < kFp8PrefetchGroups; ++g)
+      if (g < pf) quantise(g, nx[2 * g], nx[2 * g + 1]);
+#pragma unroll 4
+    for (int g = kFp8PrefetchGroups; g < groups; ++g) {
+      const int ch = 512 * g + 16 * lane;
+      quantise(g, ld16_stream(src + (size_t)ch * 2), ld16_stream(src + (size_t)ch * 2 + 16));
     }
+    prefetch(t + stride);  // in flight while this token's rows are stored
     fence_proxy_async_smem();  // these shared-memory writes before the bulk stores
     __syncwarp();
     // the scales row (H/128 floats, at most 64) by plain coalesced stores: a
