@@ -292,8 +292,14 @@ def run_reference(args, w):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.describe(), "tokens_per_step": tokens},
+        "vs_baseline": None,
+        "dtype": "fp8-e4m3 dispatch, bf16 rows, fp32 accumulate" if w.fp8 else "bf16",
+        "data": "synthetic",
+        # the same workload keys as the kernel arm's line, plus the sample size
+        "config": {"workload": w.describe(), "tokens": w.T, "hidden": w.H, "experts": w.E,
+                   "k": w.k, "ranks": w.R, "capacity": w.capacity, "rows": w.rows,
+                   "parallelism": "replicas x1 (rank 0 only)", "layout": "rows by expert, token",
+                   "router": "learned", "tokens_per_step": tokens},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
