@@ -175,6 +175,26 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def small_route_layout(T, E, k):
+    """Whether moe_route_layout runs as one cluster launch instead of the route
+    and place kernels (kSmallMaxAssign = 1024 assignments and kSmallMaxExperts
+    = 512 experts in the library's kernels.h)."""
+    return T > 0 and E <= 512 and T * k <= 1024
+
+
+def kernels_per_step(path, separate, src, small, bias_update):
+    """Kernels one step launches: route (1) + layout (count and place: 2; the
+    per-source-rank layout 4) + dispatch + combine on the separate calls; the
+    fused paths route and lay out in 2 kernels, or 1 for a small batch."""
+    if separate:
+        n = 1 + (4 if src else 2) + 2
+    elif path == "separate":
+        n = 5
+    else:
+        n = (1 if small else 2) + 2
+    return n + (1 if bias_update else 0)
+
+
 def ncu_traffic(kernel, workload):
     """Per-launch DRAM bytes from the committed ncu summary, if one exists for
     this kernel and workload (profiles/ncu_traffic.txt: `kernel workload bytes`)."""
@@ -763,9 +783,8 @@ def main():
                      "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
                      "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
                      "traffic": ncu_traffic(dom, w.name)},
-        "gpu_launches": ((7 if src else 5) if separate else
-                         {"fused3": 4, "fused": 4, "separate": 5}[args.path] + (1 if G > 0 else 0))
-                        * K,
+        "gpu_launches": kernels_per_step(args.path, separate, src,
+                                         small_route_layout(T, w.E, k), G > 0) * K,
         "clocks": clocks,
         "e2e": e2e,
     }

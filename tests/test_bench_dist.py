@@ -86,3 +86,22 @@ def test_algorithmic_bytes_cover_every_step_name():
             b = bench.algorithmic_bytes(ww, ww.rows)
             assert names <= set(b), names - set(b)
             assert all(v > 0 for v in b.values())
+
+
+def test_small_route_layout_rule_matches_the_library_constants():
+    """The bench's launch count follows the library's choice of the one-launch
+    route+layout; its limits are read from the kernel header."""
+    import re
+    import bench
+    hdr = open(os.path.join(ROOT, "combine_moe_route_07_b200", "csrc", "kernels.h")).read()
+    assign = int(re.search(r"kSmallMaxAssign = (\d+);", hdr).group(1))
+    experts = int(re.search(r"kSmallMaxExperts = (\d+);", hdr).group(1))
+    assert bench.small_route_layout(assign // 8, experts, 8)
+    assert not bench.small_route_layout(assign // 8 + 1, experts, 8)
+    assert not bench.small_route_layout(4, experts + 1, 2)
+    assert not bench.small_route_layout(0, 8, 2)
+    assert bench.kernels_per_step("fused3", False, False, True, False) == 3
+    assert bench.kernels_per_step("fused3", False, False, False, False) == 4
+    assert bench.kernels_per_step("fused3", False, False, False, True) == 5
+    assert bench.kernels_per_step("separate", False, False, True, False) == 5
+    assert bench.kernels_per_step("fused3", True, True, False, False) == 7
