@@ -385,9 +385,9 @@ cudaError_t launch_combine(const LaunchEnv& env, const void* y, const int32_t* d
   char* o = static_cast<char*>(out);
   // Dense layouts with at least 8 row slices per warp of a full bulk grid:
   // the bulk variant, when the stages of up to 12 slots (k plus the shared
-  // and residual rows) fit twice per warp.  More warps beat deeper rings:
-  // 24 warps with two stages each run the Prefill combine 2 µs faster than
-  // 16 with three; wider slices with fewer warps ran far slower.
+  // and residual rows) fit twice per warp.  Warps matter more than ring
+  // depth: 24 warps with two stages each tie or beat 16 with three, and wider
+  // slices with fewer warps ran far slower.
   const int extra = (shared != nullptr) + (residual != nullptr);
   const uint32_t stage_bytes = (uint32_t)(k + extra) * kBulkSlice;
   const int W = kBulkSmemBudget / ((size_t)kBulkMaxWarps * stage_bytes) >= 2 ? kBulkMaxWarps
