@@ -72,6 +72,12 @@ def test_reference_arm_prints_one_line_and_other_ranks_stay_silent(capsys, monke
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+    w = WORKLOADS["tiny"]
+    cfg = line["config"]
+    assert (cfg["tokens"], cfg["hidden"], cfg["experts"], cfg["k"], cfg["ranks"]) == \
+        (w.T, w.H, w.E, w.k, w.R)
+    assert cfg["rows"] == w.rows and cfg["capacity"] == w.capacity
+    assert line["metric"] == bench.METRIC and line["higher_is_better"] is True
 
 
 def test_algorithmic_bytes_cover_every_step_name():
