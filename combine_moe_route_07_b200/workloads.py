@@ -22,7 +22,12 @@ Recipe (seed 0 unless stated; one torch CPU generator, draws in this order):
   2. logits = randn(T, E) in fp32; skewed adds 2*ln(p_e) with
               p_e = (e+1)^-1.2 / sum_e' (e'+1)^-1.2 (computed in fp64, rounded
               to fp32, then one fp32 add);
-  3. bias   = rand(E) * 0.2 - 0.1 in fp32 (decode only).
+  3. bias   = rand(E) * 0.2 - 0.1 in fp32 (decode only);
+  4. shared = randn(T, H) in fp32, rounded to bf16 (workloads with a shared
+              expert): the always-on expert's output, a tensor of its own so
+              the combine's shared and residual operands differ.
+Each draw comes after the ones before it, so adding a later one leaves the
+earlier inputs unchanged.
 """
 from __future__ import annotations
 
@@ -122,6 +127,7 @@ class Inputs:
     x: torch.Tensor            # bf16 [T, H]
     logits: torch.Tensor       # fp32 [T, E]
     bias: Optional[torch.Tensor]  # fp32 [E] or None
+    shared: Optional[torch.Tensor] = None  # bf16 [T, H] shared-expert output, or None
 
 
 def zipf_offsets(E: int, s: float) -> torch.Tensor:
@@ -133,7 +139,8 @@ def zipf_offsets(E: int, s: float) -> torch.Tensor:
 
 
 def make_inputs(w: Workload, seed: Optional[int] = None) -> Inputs:
-    """Draw x, logits and bias on the CPU, in that order, from one generator."""
+    """Draw x, logits, bias and the shared-expert output on the CPU, in that
+    order, from one generator."""
     g = torch.Generator().manual_seed(w.seed if seed is None else seed)
     x = torch.randn(w.T, w.H, generator=g, dtype=torch.float32).to(torch.bfloat16)
     logits = torch.randn(w.T, w.E, generator=g, dtype=torch.float32)
@@ -142,7 +149,11 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> Inputs:
     bias = None
     if w.bias:
         bias = torch.rand(w.E, generator=g, dtype=torch.float32) * 0.2 - 0.1
-    return Inputs(x=x.contiguous(), logits=logits.contiguous(), bias=bias)
+    shared = None
+    if w.shared:
+        shared = torch.randn(w.T, w.H, generator=g, dtype=torch.float32).to(torch.bfloat16)
+        shared = shared.contiguous()
+    return Inputs(x=x.contiguous(), logits=logits.contiguous(), bias=bias, shared=shared)
 
 
 def bf16_bits(t: torch.Tensor):

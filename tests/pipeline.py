@@ -17,13 +17,17 @@ from combine_moe_route_07_b200.workloads import (WORKLOADS, Workload, bf16_bits,
 
 
 @functools.lru_cache(maxsize=2)
-def _inputs_cached(T, H, E, zipf_s, bias, seed):
-    w = Workload("tmp", T=T, H=H, E=E, R=1, k=1, zipf_s=zipf_s, bias=bias, seed=seed)
+def _inputs_cached(T, H, E, zipf_s, bias, shared, seed):
+    w = Workload("tmp", T=T, H=H, E=E, R=1, k=1, zipf_s=zipf_s, bias=bias, shared=shared,
+                 seed=seed)
     return make_inputs(w)
 
 
 def inputs_for(w: Workload):
-    return _inputs_cached(w.T, w.H, w.E, w.zipf_s, w.bias, w.seed)
+    """The workload's seeded inputs.  With a shared expert, `shared` is its own
+    draw (taken after x, logits and bias, which therefore do not change), so
+    the combine's shared and residual operands are different tensors."""
+    return _inputs_cached(w.T, w.H, w.E, w.zipf_s, w.bias, w.shared, w.seed)
 
 
 def shape_of(w: Workload):
@@ -102,8 +106,8 @@ def run_gpu(w: Workload, inp, ids=None, gates=None, fused=False):
     res["dispatch"] = disp
     y = standin_gpu(w, disp, lay)
     res["y"] = y
-    res["out"] = m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws,
-                               shared=x if w.shared else None,
+    res["shared"] = inp.shared.to(dev) if w.shared else None
+    res["out"] = m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=res["shared"],
                                residual=x if w.residual else None)
     torch.cuda.synchronize()
     return res
@@ -128,31 +132,47 @@ def run_oracle(w: Workload, inp, through="combine"):
     res["dispatch"] = disp
     y = standin_oracle(w, disp, L)
     res["y"] = y
-    res["out"] = oracle.combine(y, L["dst_pos"], gates, w.T,
-                                shared_bits=x if w.shared else None,
+    res["shared"] = bf16_bits(inp.shared) if w.shared else None
+    res["out"] = oracle.combine(y, L["dst_pos"], gates, w.T, shared_bits=res["shared"],
                                 residual_bits=x if w.residual else None)
     return res
 
 
-def oracle_combine_sampled(w: Workload, x_bits, ids, gates, dst_pos, tokens):
-    """Oracle combine for a sample of tokens, building only those tokens'
-    expert outputs (each token's k rows are its own dispatched copies)."""
+def oracle_chunk(w: Workload, x_bits, ids, gates, dst_pos, tokens, shared_bits=None):
+    """The oracle's dispatch and combine for a subset of tokens, building only
+    those tokens' rows.  Assignment (i, j) of the i-th listed token is placed
+    in local row i*k + j (its dropped slots nowhere), so the local rows hold
+    what the full dispatch writes at dst_pos[tokens[i], j]; the stand-in expert
+    then turns them into expert outputs for the combine.  shared_bits: the
+    shared-expert output of the whole batch (uint16 [T,H]) when the workload
+    has one; the residual is x.  Returns dict(keep [n,k] bool, dispatch (bf16
+    rows, or e4m3 codes and scales, local rows), out [n,H] bf16 bits)."""
     tokens = np.asarray(tokens, np.int32)
     n, k = len(tokens), w.k
     xs = x_bits[tokens]
     dp = dst_pos[tokens]
-    local = np.where(dp >= 0, np.arange(n * k, dtype=np.int32).reshape(n, k), -1).astype(np.int32)
+    keep = dp >= 0
+    local = np.where(keep, np.arange(n * k, dtype=np.int32).reshape(n, k), -1).astype(np.int32)
     if w.fp8:
-        q, s = oracle.dispatch_fp8(xs, local, n * k)
-        y = oracle.dequant_fp8(q, s)
+        disp = oracle.dispatch_fp8(xs, local, n * k)
+        y = oracle.dequant_fp8(*disp)
     else:
-        y = oracle.dispatch_bf16(xs, local, n * k)
+        disp = oracle.dispatch_bf16(xs, local, n * k)
+        y = disp
         if w.expert == "scale":
             y = _scale_rows(w, y, ids[tokens].reshape(-1).astype(np.int32))
-    out = oracle.combine(y, local, gates[tokens], n,
-                         shared_bits=xs if w.shared else None,
+    sh = None
+    if w.shared:
+        assert shared_bits is not None, "the workload has a shared expert: pass its output"
+        sh = shared_bits[tokens]
+    out = oracle.combine(y, local, gates[tokens], n, shared_bits=sh,
                          residual_bits=xs if w.residual else None)
-    return out
+    return {"keep": keep, "dispatch": disp, "out": out}
+
+
+def oracle_combine_sampled(w: Workload, x_bits, ids, gates, dst_pos, tokens, shared_bits=None):
+    """Oracle combine for a sample of tokens (see oracle_chunk)."""
+    return oracle_chunk(w, x_bits, ids, gates, dst_pos, tokens, shared_bits)["out"]
 
 
 def _scale_rows(w, y, e_of_row):

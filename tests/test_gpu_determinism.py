@@ -24,7 +24,8 @@ def _path(w, inp, dev):
     ids, gates, lay = m.moe_route_layout(shape, inp.logits.to(dev), bias, ws=ws)
     xd = m.moe_dispatch(shape, x, lay.dst_pos, ws=ws)
     y = xd if not w.fp8 else (xd[0].float() * xd[1].repeat_interleave(128, dim=1)).to(torch.bfloat16)
-    out = m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=x if w.shared else None,
+    shared = inp.shared.to(dev) if w.shared else None
+    out = m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared,
                         residual=x if w.residual else None)
     torch.cuda.synchronize()
     assert m.moe_get_device_error(ws) == (0, 0)

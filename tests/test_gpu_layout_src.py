@@ -155,7 +155,8 @@ def test_dispatch_and_combine_over_the_src_layout(capacity_factor):
     e_of_row = np.where(src >= 0, ids_np.ravel()[np.maximum(src, 0)], 0)
     scale = ((torch.arange(1, w.E + 1, dtype=torch.float32) / float(w.E))[e_of_row]).to(dev)
     y = (xd.float() * scale[:, None]).to(torch.bfloat16)
-    out = m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=x, residual=x)
+    sh = inp.shared.to(dev)  # the shared expert's output: its own draw, not x
+    out = m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=sh, residual=x)
     torch.cuda.synchronize()
     assert m.moe_get_device_error(ws) == (0, 0)
 
@@ -167,6 +168,6 @@ def test_dispatch_and_combine_over_the_src_layout(capacity_factor):
     assert np.array_equal(to_np(xd).view(np.uint16)[used], rows[used])
     # the combine over the same expert rows the GPU combined (the stand-in
     # expert is outside the path)
-    want = oracle.combine(to_np(y), o["dst_pos"], to_np(gates), w.T, shared_bits=xb,
-                          residual_bits=xb)
+    want = oracle.combine(to_np(y), o["dst_pos"], to_np(gates), w.T,
+                          shared_bits=bf16_bits(inp.shared), residual_bits=xb)
     assert_bf16_close(to_np(out), want, 1, "src_path")
