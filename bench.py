@@ -17,7 +17,11 @@ the event intervals.
 
 Prints ONE JSON line (rank 0).  With N > 1 (torchrun, one process per GPU)
 every rank runs its own batch (weak scaling, no collective on the data path);
-the reported time is the max over ranks.
+the reported time is the max over ranks.  On one GPU the line also carries a
+`per_workload` block: the other workloads (tiny, decode, skewed with capacity
+and dropless, fine-grained) each measured the same way with fewer steps, and
+a `cpu_baseline` (the oracle on this host, with its core count, CPU model and
+per-stage times).  Both arms print the same `config` object.
 """
 import argparse
 import json
@@ -36,7 +40,7 @@ FALLBACK_HBM_GBS = 6650.0
 METRIC = "dispatch+combine tokens/s at 1 B200; achieved HBM GB/s vs peak"
 
 
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=3000)
@@ -70,7 +74,12 @@ def parse():
     p.add_argument("--path", choices=["fused3", "fused", "separate"], default="fused3",
                    help="steps 1-4 in one moe_route_layout_dispatch call; route+layout in one "
                         "moe_route_layout call; or one call per step")
-    return p.parse_args()
+    p.add_argument("--per-workload", default="tiny,decode,skewed_capacity,skewed_dropless,"
+                                             "finegrained",
+                   help="comma-separated workloads also measured (one GPU only) and reported "
+                        "in the line's per_workload block; 'none' for none")
+    p.add_argument("--per-workload-steps", type=int, default=50)
+    return p.parse_args(argv)
 
 
 # ------------------------------------------------------------ byte counts --
@@ -230,13 +239,37 @@ def whole_job_tokens_per_s(world: int, tokens_per_rank: int, steps: int, max_ms:
 
 # ----------------------------------------------------------------- oracle --
 
+def host_facts():
+    """The host the oracle runs on: logical CPUs, the ones this process may
+    use, and the CPU model string."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        usable = os.cpu_count()
+    return {"host_cores": os.cpu_count(), "usable_cores": usable, "cpu_model": model}
+
+
+STAGES = ("route", "layout", "dispatch", "combine")
+
+
 def oracle_step_fn(w, inp, tokens):
-    """One oracle pass of the path over the first `tokens` tokens (expert
-    output prepared outside the returned closure)."""
+    """One oracle pass of the path over the first `tokens` tokens (the expert
+    output is prepared outside the returned closure, which returns the seconds
+    each stage took)."""
     import numpy as np
     import oracle
     from combine_moe_route_07_b200.workloads import bf16_bits
     x = np.ascontiguousarray(bf16_bits(inp.x)[:tokens])
+    sh = np.ascontiguousarray(bf16_bits(inp.shared)[:tokens]) if w.shared else None
     logits = np.ascontiguousarray(inp.logits.numpy()[:tokens])
     bias = None if inp.bias is None else inp.bias.numpy()
     cap = w.capacity if w.capacity == 0 else max(1, -(-w.capacity * tokens // w.T))
@@ -252,35 +285,103 @@ def oracle_step_fn(w, inp, tokens):
             if w.expert == "scale" else d
 
     def step():
+        t = [time.perf_counter()]
         i2, g2 = oracle.route(logits, w.k, bias, renorm=w.renorm)
+        t.append(time.perf_counter())
         L2 = oracle.layout(i2, w.E, w.R, capacity=cap, align=w.align)
+        t.append(time.perf_counter())
         if w.fp8:
             oracle.dispatch_fp8(x, L2["dst_pos"], N)
         else:
             oracle.dispatch_bf16(x, L2["dst_pos"], N)
-        oracle.combine(y, L2["dst_pos"], g2, tokens, shared_bits=x if w.shared else None,
+        t.append(time.perf_counter())
+        oracle.combine(y, L2["dst_pos"], g2, tokens, shared_bits=sh,
                        residual_bits=x if w.residual else None)
+        t.append(time.perf_counter())
+        return [b - a for a, b in zip(t, t[1:])]
     return step
 
 
 def time_oracle(w, inp, budget_s, max_steps=None):
     """Time the oracle on a bounded sample: the whole batch if one pass fits
-    the budget, else a prefix of tokens; returns (tokens/s, sample text)."""
+    the budget, else a prefix of tokens.  Returns (tokens/s, tokens, passes,
+    seconds, per-stage milliseconds of one pass)."""
     tokens = w.T
     step = oracle_step_fn(w, inp, tokens)
-    t0 = time.perf_counter()
-    step()
-    one = time.perf_counter() - t0
+    one = sum(step())
     if one > budget_s and tokens > 1:
         tokens = max(1, int(tokens * budget_s / one / 2))
         step = oracle_step_fn(w, inp, tokens)
     reps, elapsed = 0, 0.0
+    stage = [0.0] * len(STAGES)
     while elapsed < budget_s and (max_steps is None or reps < max_steps):
-        t0 = time.perf_counter()
-        step()
-        elapsed += time.perf_counter() - t0
+        st = step()
+        stage = [a + b for a, b in zip(stage, st)]
+        elapsed += sum(st)
         reps += 1
-    return tokens * reps / elapsed, tokens, reps, elapsed
+    stage_ms = {n: round(v / reps * 1e3, 3) for n, v in zip(STAGES, stage)}
+    return tokens * reps / elapsed, tokens, reps, elapsed, stage_ms
+
+
+# ------------------------------------------------------------ the step plan --
+
+def step_plan(w, args):
+    """The calls one step makes, in order, and whether route and layout are
+    separate calls because a variant asks for them (no device work here)."""
+    src = args.layout == "src"
+    M, RR, HOME, G = args.max_ranks, args.router == "round_robin", args.home, args.bias_gamma
+    separate = src or M > 0 or RR or HOME >= 0
+    if separate:
+        names = ["route_round_robin" if RR else ("route_limited" if M > 0 else "route"),
+                 "layout_src" if src else ("layout_remote_first" if HOME >= 0 else "layout"),
+                 "dispatch", "combine"]
+    elif args.path == "fused3":
+        names = ["route_layout_dispatch", "combine"]
+    elif args.path == "fused":
+        names = ["route_layout", "dispatch", "combine"]
+    else:
+        names = ["route", "layout", "dispatch", "combine"]
+    if G > 0:
+        names.insert(names.index("combine"), "bias_update")
+    return tuple(names), separate
+
+
+L2_BYTES = 126 * 10**6
+
+
+def touched_bytes(w, args, kept_rows):
+    b = algorithmic_bytes(w, kept_rows)
+    lay = "layout_src" if args.layout == "src" else "layout"
+    return b["route"] + b[lay] + b["dispatch"] + b["combine"]
+
+
+def flushes_between_steps(w, args):
+    """Whether the steps are separated by an L2 flush: when a step touches
+    less than twice the L2 (counted at the layout's static row count)."""
+    return touched_bytes(w, args, w.rows) < 2 * L2_BYTES
+
+
+def bench_config(w, args, world):
+    """The `config` object of the JSON line; both arms print this same object."""
+    names, _ = step_plan(w, args)
+    src = args.layout == "src"
+    touched = touched_bytes(w, args, w.rows)
+    return {
+        "workload": w.describe(), "tokens": w.T, "hidden": w.H, "experts": w.E, "k": w.k,
+        "ranks": w.R, "capacity": w.capacity_src if src else w.capacity,
+        "rows": w.rows_src if src else w.rows, "parallelism": f"replicas x{world}",
+        "l2": ("256 MiB write + read between timed steps, outside the step events"
+               if flushes_between_steps(w, args) else
+               f"no flush: inputs larger than L2 ({touched / 1e6:.0f} MB touched per step vs "
+               f"126 MB L2), steps back to back"),
+        "layout": ("per-source-rank: rows by destination rank, source shard (R shards of "
+                   "ceil(T/R) tokens), expert, token") if src else "rows by expert, token",
+        "max_ranks": args.max_ranks if args.max_ranks > 0 else None,
+        "bias_gamma": args.bias_gamma if args.bias_gamma > 0 else None,
+        "router": args.router,
+        "home_rank": args.home if args.home >= 0 else None,
+        "step": " + ".join(names) + ", one CUDA graph",
+    }
 
 
 def run_reference(args, w):
@@ -294,20 +395,19 @@ def run_reference(args, w):
     # sized so that the timed steps take about a minute in all
     probe_tokens = max(1, w.T // 16)
     step = oracle_step_fn(w, inp, probe_tokens)
-    t0 = time.perf_counter()
-    step()
-    per_token = (time.perf_counter() - t0) / probe_tokens
+    per_token = sum(step()) / probe_tokens
     budget = 60.0 / max(1, args.steps + args.warmup)
     tokens = int(min(w.T, max(8, budget / per_token)))
     step = oracle_step_fn(w, inp, tokens)
     for _ in range(args.warmup):
         step()
-    t0 = time.perf_counter()
+    stage = [0.0] * len(STAGES)
     for _ in range(args.steps):
-        step()
-    el = time.perf_counter() - t0
+        stage = [a + b for a, b in zip(stage, step())]
+    el = sum(stage)
     value = tokens * args.steps / el
     sample = f"first {tokens} of {w.T} tokens of the {w.name} batch per step, single thread"
+    world = int(os.environ.get("WORLD_SIZE", str(getattr(args, "gpus", 1))))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -315,13 +415,12 @@ def run_reference(args, w):
         "vs_baseline": None,
         "dtype": "fp8-e4m3 dispatch, bf16 rows, fp32 accumulate" if w.fp8 else "bf16",
         "data": "synthetic",
-        # the same workload keys as the kernel arm's line, plus the sample size
-        "config": {"workload": w.describe(), "tokens": w.T, "hidden": w.H, "experts": w.E,
-                   "k": w.k, "ranks": w.R, "capacity": w.capacity, "rows": w.rows,
-                   "parallelism": "replicas x1 (rank 0 only)", "layout": "rows by expert, token",
-                   "router": "learned", "tokens_per_step": tokens},
+        "config": bench_config(w, args, world),
+        "tokens_per_step": tokens,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, **host_facts(),
+                         "stage_ms_per_step": {n: round(v / args.steps * 1e3, 3)
+                                               for n, v in zip(STAGES, stage)}},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -330,6 +429,282 @@ def run_reference(args, w):
 
 
 # ----------------------------------------------------------------- native --
+
+class Path:
+    """Device buffers and the calls of one step of one workload (the library's
+    public API, torch only for memory and streams)."""
+
+    def __init__(self, args, w, dev, seed):
+        import torch
+        import combine_moe_route_07_b200 as m
+        from combine_moe_route_07_b200.workloads import make_inputs
+        self.m, self.args, self.w, self.dev = m, args, w, dev
+        self.inp = inp = make_inputs(w, seed=seed)
+        src = self.src = args.layout == "src"
+        shape = self.shape = m.MoeShape(
+            tokens=w.T, hidden=w.H, experts=w.E, k=w.k, ranks=w.R,
+            capacity=w.capacity_src if src else w.capacity, align=w.align, renorm=w.renorm,
+            fp8=w.fp8, src_layout=src)
+        ws = self.ws = m.Workspace(shape, dev)
+        self.x = inp.x.to(dev)
+        self.logits = inp.logits.to(dev)
+        bias = None if inp.bias is None else inp.bias.to(dev)
+        G = args.bias_gamma
+        if G > 0 and bias is None:
+            bias = torch.zeros(w.E, dtype=torch.float32, device=dev)
+        self.bias = bias
+        # the shared expert's output: a tensor of its own (not x), read by the combine
+        self.shared = inp.shared.to(dev) if w.shared else None
+        T, k, N = w.T, w.k, shape.rows
+        i32 = dict(dtype=torch.int32, device=dev)
+        ids = self.ids = torch.empty((T, k), **i32)
+        gates = self.gates = torch.empty((T, k), dtype=torch.float32, device=dev)
+        if src:
+            lay = m.LayoutSrc(torch.empty((w.R, w.E), **i32), torch.empty(w.R * w.E + 1, **i32),
+                              torch.empty((w.R, w.R), **i32), torch.empty(w.R + 1, **i32),
+                              torch.empty(w.R, **i32), torch.empty((T, k), **i32),
+                              torch.empty(N, **i32))
+        else:
+            lay = m.Layout(torch.empty(w.E, **i32), torch.empty(w.E + 1, **i32),
+                           torch.empty(w.R + 1, **i32), torch.empty(w.R, **i32),
+                           torch.empty((T, k), **i32), torch.empty(N, **i32))
+        self.lay = lay
+        if w.fp8:
+            xd = torch.empty((N, w.H), dtype=torch.float8_e4m3fn, device=dev)
+            sc = torch.empty((N, w.H // 128), dtype=torch.float32, device=dev)
+        else:
+            xd = torch.empty((N, w.H), dtype=torch.bfloat16, device=dev)
+            sc = None
+        self.xd, self.sc = xd, sc
+        self.out = torch.empty((T, w.H), dtype=torch.bfloat16, device=dev)
+        M, RR, HOME = args.max_ranks, args.router == "round_robin", args.home
+        tile_expert = (torch.empty(N // w.align, dtype=torch.int32, device=dev) if HOME >= 0
+                       else None)
+
+        def route():
+            if RR:
+                m.moe_route_round_robin(shape, ids=ids, gates=gates)
+            elif M > 0:
+                m.moe_route_limited(shape, self.logits, M, bias, ws=ws, ids=ids, gates=gates)
+            else:
+                m.moe_route(shape, self.logits, bias, ws=ws, ids=ids, gates=gates)
+
+        def layout():
+            if src:
+                m.moe_layout_src(shape, ids, ws=ws, out=lay)
+            elif HOME >= 0:
+                m.moe_layout_remote_first(shape, ids, HOME, ws=ws, out=lay,
+                                          tile_expert=tile_expert)
+            else:
+                m.moe_layout(shape, ids, ws=ws, out=lay)
+
+        def dispatch():
+            m.moe_dispatch(shape, self.x, lay.dst_pos, ws=ws, out=xd, scales=sc)
+
+        def combine():
+            m.moe_combine(shape, self.y, lay.dst_pos, gates, ws=ws, shared=self.shared,
+                          residual=self.x if w.residual else None, out=self.out)
+
+        calls = {
+            "route": route, "route_limited": route, "route_round_robin": route,
+            "layout": layout, "layout_src": layout, "layout_remote_first": layout,
+            "route_layout": lambda: m.moe_route_layout(shape, self.logits, bias, ws=ws, ids=ids,
+                                                       gates=gates, out=lay),
+            "route_layout_dispatch": lambda: m.moe_route_layout_dispatch(
+                shape, self.logits, self.x, bias, ws=ws, ids=ids, gates=gates, lay=lay, out=xd,
+                scales=sc),
+            "dispatch": dispatch, "combine": combine,
+            "bias_update": lambda: m.moe_bias_update(shape, lay.counts, G, bias),
+        }
+        self.names, self.separate = step_plan(w, args)
+        self.ops = [calls[n] for n in self.names]
+        # the per-kernel probe splits the fused steps 1-4 at the dispatch
+        if self.names[0] == "route_layout_dispatch":
+            self.probe_names = ("route_layout", "dispatch") + self.names[1:]
+        else:
+            self.probe_names = self.names
+        self.probe_ops = [calls[n] for n in self.probe_names]
+        self.calls = calls
+
+        # the expert stand-in's output for this batch, prepared once (outside the path)
+        route()
+        layout()
+        dispatch()
+        if w.fp8:
+            y = (xd.float() * sc.repeat_interleave(128, dim=1)).to(torch.bfloat16)
+        elif w.expert == "scale":
+            # expert of every row from src_idx (any row order); empty rows read expert 0
+            e = ids.flatten()[lay.src_idx.clamp(min=0).long()].long()
+            s = (torch.arange(1, w.E + 1, dtype=torch.float32, device=dev)
+                 / torch.tensor(float(w.E), device=dev))[e]
+            y = (xd.float() * s[:, None]).to(torch.bfloat16)
+        else:
+            y = xd.clone()
+        self.y = y
+        torch.cuda.synchronize()
+        self.kept_rows = int(lay.rank_counts.sum().item())
+        m.moe_check(ws)
+
+    def step(self):
+        for op in self.ops:
+            op()
+
+    def m_check(self):
+        """Raise if a kernel recorded a device-side error."""
+        self.m.moe_check(self.ws)
+
+
+def _flush_fn(buf):
+    """An L2 flush (a 256 MiB write, then a read that leaves L2 clean), or a
+    no-op when buf is None."""
+    import torch
+
+    def flush():
+        if buf is not None:
+            buf.fill_(1)
+            buf.view(torch.int64).sum()
+    return flush
+
+
+def capture_step(path, warmup, stream, flush):
+    """Warm up eagerly, then capture the step as one CUDA graph: the step is
+    launch-bound at its small kernels, and a graph replay is how the path is
+    meant to be driven."""
+    import torch
+    dev = path.dev
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for _ in range(max(3, warmup)):
+            flush()
+            path.step()
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        path.step()
+    for _ in range(3):
+        flush()
+        g.replay()
+    torch.cuda.synchronize()
+    path.m_check()
+    return g
+
+
+def time_steps(g, K, stream, flush):
+    """Per-step CUDA-event times (ms) of K graph replays, the L2 flush (when
+    used) outside the events."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    for i in range(K):
+        flush()
+        ev[i][0].record(stream)
+        g.replay()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def probe_kernels(path, K_ops, flush):
+    """Per-call device time inside the step: a probe graph of the same step
+    with event-record nodes between the calls, replayed after an L2 flush and
+    read back one replay at a time; the mean over K_ops replays."""
+    import torch
+    dev = path.dev
+    n = len(path.probe_ops)
+    pev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n + 1)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        cap = torch.cuda.current_stream(dev)
+        pev[0].record(cap)
+        for j, op in enumerate(path.probe_ops):
+            op()
+            pev[j + 1].record(cap)
+    sums = [0.0] * n
+    for _ in range(K_ops):
+        flush()
+        g.replay()
+        torch.cuda.synchronize()
+        for j in range(n):
+            sums[j] += pev[j].elapsed_time(pev[j + 1])
+    del g
+    return [v / K_ops for v in sums]
+
+
+def time_isolated(path, K_ops, iso_buf, stream):
+    """Dispatch and combine each on its own: a 256 MiB L2 write + read-back
+    before every launch (outside the events, so the dirty lines of the
+    previous op are written back there); the median over K_ops launches."""
+    import torch
+    iso = {}
+    for name in ("dispatch", "combine"):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            path.calls[name]()
+        times = []
+        for _ in range(K_ops):
+            iso_buf.fill_(1)
+            iso_buf.view(torch.int64).sum()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        del g
+        iso[name] = sorted(times)[len(times) // 2]
+    return iso
+
+
+def dc_summary(w, kept_rows, t_disp, t_comb, peak):
+    """Dispatch + combine: µs, GB/s and the fractions of the measured copy
+    peak and of 8 TB/s, from the two ops' times in ms."""
+    b = algorithmic_bytes(w, kept_rows)
+    ms = t_disp + t_comb
+    gbs = (b["dispatch"] + b["combine"]) / (ms * 1e-3) / 1e9
+    return {"us": round(ms * 1e3, 2), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+            "frac_of_8tbs": round(gbs / 8000.0, 4)}
+
+
+def measure_workload(args, w, dev, stream, peak, K, warmup):
+    """A compact measurement of one more workload (one GPU): the step as one
+    graph replayed K times, per-call times inside the step, and dispatch and
+    combine each alone after an L2 flush."""
+    import torch
+    path = Path(args, w, dev, seed=w.seed)
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = _flush_fn(flush_buf if flushes_between_steps(w, args) else None)
+    g = capture_step(path, warmup, stream, flush)
+    times = time_steps(g, K, stream, flush)
+    del g
+    K_ops = 20
+    mean = probe_kernels(path, K_ops, flush)
+    iso = time_isolated(path, K_ops, flush_buf, stream)
+    path.m_check()
+    byts = algorithmic_bytes(w, path.kept_rows)
+    ms = sum(times) / K
+    t_disp = mean[path.probe_names.index("dispatch")]
+    t_comb = mean[path.probe_names.index("combine")]
+    kern = {}
+    for s, name in enumerate(path.probe_names):
+        gbs = byts[name] / (mean[s] * 1e-3) / 1e9
+        kern[name] = {"us": round(mean[s] * 1e3, 2), "frac": round(gbs / peak, 4)}
+    res = {
+        "workload": w.describe(), "steps": K, "us_per_step": round(ms * 1e3, 2),
+        "tokens_per_s": w.T / (ms * 1e-3), "rows": path.shape.rows,
+        "kept_rows": path.kept_rows,
+        "l2": "flushed between steps" if flushes_between_steps(w, args) else "steps back to back",
+        "dispatch_combine_in_step": dc_summary(w, path.kept_rows, t_disp, t_comb, peak),
+        "dispatch_combine_isolated": dc_summary(w, path.kept_rows, iso["dispatch"],
+                                                iso["combine"], peak),
+        "kernels_in_step": kern,
+    }
+    del path, flush_buf
+    torch.cuda.empty_cache()
+    return res
+
 
 def main():
     args = parse()
@@ -355,182 +730,18 @@ def main():
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-
-    import combine_moe_route_07_b200 as m
-    from combine_moe_route_07_b200.workloads import make_inputs
-
-    inp = make_inputs(w, seed=w.seed + rank)
-    src = args.layout == "src"
-    shape = m.MoeShape(tokens=w.T, hidden=w.H, experts=w.E, k=w.k, ranks=w.R,
-                       capacity=w.capacity_src if src else w.capacity, align=w.align,
-                       renorm=w.renorm, fp8=w.fp8, src_layout=src)
-    ws = m.Workspace(shape, dev)
-    x = inp.x.to(dev)
-    logits = inp.logits.to(dev)
-    bias = None if inp.bias is None else inp.bias.to(dev)
-    G = args.bias_gamma
-    if G > 0 and bias is None:
-        bias = torch.zeros(w.E, dtype=torch.float32, device=dev)
-    T, k, N = w.T, w.k, shape.rows
-    i32 = dict(dtype=torch.int32, device=dev)
-    ids = torch.empty((T, k), **i32)
-    gates = torch.empty((T, k), dtype=torch.float32, device=dev)
-    if src:
-        lay = m.LayoutSrc(torch.empty((w.R, w.E), **i32), torch.empty(w.R * w.E + 1, **i32),
-                          torch.empty((w.R, w.R), **i32), torch.empty(w.R + 1, **i32),
-                          torch.empty(w.R, **i32), torch.empty((T, k), **i32),
-                          torch.empty(N, **i32))
-    else:
-        lay = m.Layout(torch.empty(w.E, **i32), torch.empty(w.E + 1, **i32),
-                       torch.empty(w.R + 1, **i32), torch.empty(w.R, **i32),
-                       torch.empty((T, k), **i32), torch.empty(N, **i32))
-    if w.fp8:
-        xd = torch.empty((N, w.H), dtype=torch.float8_e4m3fn, device=dev)
-        sc = torch.empty((N, w.H // 128), dtype=torch.float32, device=dev)
-    else:
-        xd = torch.empty((N, w.H), dtype=torch.bfloat16, device=dev)
-        sc = None
-    out = torch.empty((T, w.H), dtype=torch.bfloat16, device=dev)
-    shared = x if w.shared else None
-    residual = x if w.residual else None
-
-    M = args.max_ranks
-
-    RR = args.router == "round_robin"
-    HOME = args.home
-
-    def route_op():
-        if RR:
-            m.moe_route_round_robin(shape, ids=ids, gates=gates)
-        elif M > 0:
-            m.moe_route_limited(shape, logits, M, bias, ws=ws, ids=ids, gates=gates)
-        else:
-            m.moe_route(shape, logits, bias, ws=ws, ids=ids, gates=gates)
-
-    tile_expert = (torch.empty(N // w.align, dtype=torch.int32, device=dev) if HOME >= 0
-                   else None)
-
-    def layout_op():
-        if src:
-            m.moe_layout_src(shape, ids, ws=ws, out=lay)
-        elif HOME >= 0:
-            m.moe_layout_remote_first(shape, ids, HOME, ws=ws, out=lay, tile_expert=tile_expert)
-        else:
-            m.moe_layout(shape, ids, ws=ws, out=lay)
-
-    def route_layout_dispatch():
-        route_op()
-        layout_op()
-        m.moe_dispatch(shape, x, lay.dst_pos, ws=ws, out=xd, scales=sc)
-
-    # the expert stand-in's output for this batch, prepared once
-    route_layout_dispatch()
-    if w.fp8:
-        y = (xd.float() * sc.repeat_interleave(128, dim=1)).to(torch.bfloat16)
-    elif w.expert == "scale":
-        # expert of every row from src_idx (any row order); empty rows read expert 0
-        e = ids.flatten()[lay.src_idx.clamp(min=0).long()].long()
-        s = (torch.arange(1, w.E + 1, dtype=torch.float32, device=dev)
-             / torch.tensor(float(w.E), device=dev))[e]
-        y = (xd.float() * s[:, None]).to(torch.bfloat16)
-    else:
-        y = xd.clone()
-    torch.cuda.synchronize()
-    kept_rows = int(lay.rank_counts.sum().item())
-    m.moe_check(ws)
-
-    L2_BYTES = 126 * 10**6
-    _b = algorithmic_bytes(w, kept_rows)
-    touched = _b["route"] + _b["layout_src" if src else "layout"] + _b["dispatch"] + _b["combine"]
-    flush_between = touched < 2 * L2_BYTES
-    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush_between else None
-
-    def flush():
-        if flush_between:
-            flush_buf.fill_(1)
-            flush_buf.view(torch.int64).sum()  # read it back: L2 left clean
-
     stream = torch.cuda.current_stream(dev)
+    import combine_moe_route_07_b200 as m
 
-    names_probe = ("route_layout", "dispatch", "combine")
-    ops_probe = (
-        lambda: m.moe_route_layout(shape, logits, bias, ws=ws, ids=ids, gates=gates, out=lay),
-        lambda: m.moe_dispatch(shape, x, lay.dst_pos, ws=ws, out=xd, scales=sc),
-        lambda: m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared,
-                              residual=residual, out=out),
-    )
-    bias_op = lambda: m.moe_bias_update(shape, lay.counts, G, bias)  # noqa: E731
-    if G > 0:
-        names_probe = ("route_layout", "dispatch", "bias_update", "combine")
-        ops_probe = (ops_probe[0], ops_probe[1], bias_op, ops_probe[2])
-    if src or M > 0 or RR or HOME >= 0:
-        names = ("route_round_robin" if RR else ("route_limited" if M > 0 else "route"),
-                 "layout_src" if src else ("layout_remote_first" if HOME >= 0 else "layout"),
-                 "dispatch", "combine")
-        ops = (
-            route_op,
-            layout_op,
-            lambda: m.moe_dispatch(shape, x, lay.dst_pos, ws=ws, out=xd, scales=sc),
-            lambda: m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared,
-                                  residual=residual, out=out),
-        )
-    elif args.path == "fused3":
-        names = ("route_layout_dispatch", "combine")
-        ops = (
-            lambda: m.moe_route_layout_dispatch(shape, logits, x, bias, ws=ws, ids=ids, gates=gates,
-                                                lay=lay, out=xd, scales=sc),
-            lambda: m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared,
-                                  residual=residual, out=out),
-        )
-        if G > 0:
-            names = ("route_layout_dispatch", "bias_update", "combine")
-            ops = (ops[0], bias_op, ops[1])
-    elif args.path == "fused":
-        names = ("route_layout", "dispatch", "combine")
-        ops = (
-            lambda: m.moe_route_layout(shape, logits, bias, ws=ws, ids=ids, gates=gates,
-                                       out=lay),
-            lambda: m.moe_dispatch(shape, x, lay.dst_pos, ws=ws, out=xd, scales=sc),
-            lambda: m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared,
-                                  residual=residual, out=out),
-        )
-    else:
-        names = ("route", "layout", "dispatch", "combine")
-        ops = (
-            lambda: m.moe_route(shape, logits, bias, ws=ws, ids=ids, gates=gates),
-            lambda: m.moe_layout(shape, ids, ws=ws, out=lay),
-            lambda: m.moe_dispatch(shape, x, lay.dst_pos, ws=ws, out=xd, scales=sc),
-            lambda: m.moe_combine(shape, y, lay.dst_pos, gates, ws=ws, shared=shared,
-                                  residual=residual, out=out),
-        )
+    path = Path(args, w, dev, seed=w.seed + rank)
+    T, k, N = w.T, w.k, path.shape.rows
+    kept_rows = path.kept_rows
+    flush_between = flushes_between_steps(w, args)
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = _flush_fn(flush_buf if flush_between else None)
 
-    def step():
-        for op in ops:
-            op()
-
-    # warm up eagerly, then capture the step (and each op on its own) as CUDA
-    # graphs: the step is launch-bound at its small kernels, and a graph replay
-    # is how the path is meant to be driven
-    side = torch.cuda.Stream(dev)
-    side.wait_stream(stream)
-    with torch.cuda.stream(side):
-        for _ in range(max(3, args.warmup)):
-            flush()
-            step()
-    stream.wait_stream(side)
-    torch.cuda.synchronize()
-    g_step = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_step):
-        step()
-    for _ in range(3):
-        flush()
-        g_step.replay()
-    torch.cuda.synchronize()
-    m.moe_check(ws)
-
+    g_step = capture_step(path, args.warmup, stream, flush)
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
     sampler = ClockSampler(local) if rank == 0 else None
     if dist is not None:
         dist.barrier()
@@ -538,70 +749,18 @@ def main():
     if sampler:
         sampler.start()
         time.sleep(0.3)
-    for i in range(K):
-        flush()
-        ev[i][0].record(stream)
-        g_step.replay()
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
+    times = time_steps(g_step, K, stream, flush)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
-    m.moe_check(ws)
-    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dist, dev)
+    m.moe_check(path.ws)
+    total_ms = max_over_ranks(sum(times), dist, dev)
+    del g_step
 
-    # per-kernel breakdown: a probe graph of the same step with event-record
-    # nodes between the kernels, replayed after an L2 flush and read back one
-    # replay at a time
-    separate = src or M > 0 or RR or HOME >= 0
-    probe_names = names if (separate or args.path != "fused3") else names_probe
-    probe_ops = ops if (separate or args.path != "fused3") else ops_probe
-    n_ops = len(probe_ops)
-    probe_ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ops + 1)]
-    g_probe = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_probe):
-        cap = torch.cuda.current_stream(dev)
-        probe_ev[0].record(cap)
-        for j, op in enumerate(probe_ops):
-            op()
-            probe_ev[j + 1].record(cap)
     K_ops = max(20, min(400, K // 10))
-    sums = [0.0] * n_ops
-    for i in range(K_ops):
-        flush()
-        g_probe.replay()
-        torch.cuda.synchronize()
-        for j in range(n_ops):
-            sums[j] += probe_ev[j].elapsed_time(probe_ev[j + 1])
-    mean = [v / K_ops for v in sums]
-    del g_probe
-
-    # dispatch and combine each on its own: a 256 MiB L2 write + read-back
-    # before every launch (outside the events, so dirty lines of the previous
-    # op are written back there), median over the iterations
-    iso_buf = flush_buf if flush_buf is not None else torch.empty(256 << 20, dtype=torch.uint8,
-                                                                  device=dev)
-    iso = {}
-    for name in ("dispatch", "combine"):
-        op = ops_probe[names_probe.index(name)]
-        g_op = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_op):
-            op()
-        times = []
-        for i in range(K_ops):
-            iso_buf.fill_(1)
-            iso_buf.view(torch.int64).sum()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            g_op.replay()
-            b.record(stream)
-            torch.cuda.synchronize()
-            times.append(a.elapsed_time(b))
-        del g_op
-        iso[name] = sorted(times)[len(times) // 2]
-    iso_n = K_ops
+    mean = probe_kernels(path, K_ops, flush)
+    iso = time_isolated(path, K_ops, flush_buf, stream)
 
     # the achievable floor for the same bytes: a plain device-to-device copy
     # moving as many bytes (read + write) as dispatch and combine together,
@@ -612,9 +771,9 @@ def main():
     cdst = torch.empty_like(csrc)
     csrc.fill_(3)
     ctimes = []
-    for i in range(K_ops):
-        iso_buf.fill_(1)
-        iso_buf.view(torch.int64).sum()
+    for _ in range(K_ops):
+        flush_buf.fill_(1)
+        flush_buf.view(torch.int64).sum()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -623,7 +782,7 @@ def main():
         torch.cuda.synchronize()
         ctimes.append(a.elapsed_time(b))
     copy_ms = sorted(ctimes)[len(ctimes) // 2]
-    del csrc, cdst, iso_buf
+    del csrc, cdst
 
     # end to end through the public API: every step copies its inputs in from
     # pinned host memory and its result back out.  Pipelined the way a server
@@ -634,19 +793,20 @@ def main():
     # replayed, so host launch overhead does not stand in for the copies.
     e2e = None
     if args.e2e_steps > 0:
+        inp = path.inp
         x_h = inp.x.pin_memory()
         lg_h = inp.logits.pin_memory()
         out_h = [torch.empty((T, w.H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-        set_a = (x, logits, out)
-        set_b = (torch.empty_like(x), torch.empty_like(logits), torch.empty_like(out))
+        set_a = (path.x, path.logits, path.out)
+        set_b = (torch.empty_like(path.x), torch.empty_like(path.logits),
+                 torch.empty_like(path.out))
         sets = (set_a, set_b)
-
         U = 64
         cin, cout = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        x, logits, out = set_b
-        shared = x if w.shared else None
-        residual = x if w.residual else None
-        step()  # the second set's first pass, outside capture
+        path.x, path.logits, path.out = set_b
+        set_b[0].copy_(path.inp.x)
+        set_b[1].copy_(path.inp.logits)
+        path.step()  # the second set's first pass, outside capture
         torch.cuda.synchronize()
         g_e2e = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_e2e):
@@ -667,10 +827,8 @@ def main():
                 cap.wait_event(h2d_e)
                 if u >= 2:
                     cap.wait_event(evs[u - 2][2])  # step u-2's result has left this set
-                x, logits, out = xs, ls, os_
-                shared = x if w.shared else None
-                residual = x if w.residual else None
-                step()
+                path.x, path.logits, path.out = xs, ls, os_
+                path.step()
                 done_e.record(cap)
                 with torch.cuda.stream(cout):
                     cout.wait_event(done_e)
@@ -679,9 +837,7 @@ def main():
                 evs.append((h2d_e, done_e, d2h_e))
             cap.wait_stream(cin)
             cap.wait_stream(cout)
-        x, logits, out = set_a
-        shared = x if w.shared else None
-        residual = x if w.residual else None
+        path.x, path.logits, path.out = set_a
         reps = max(1, -(-args.e2e_steps // U))
         for _ in range(2):
             g_e2e.replay()
@@ -702,6 +858,7 @@ def main():
                "mode": ("pipelined over two buffer sets: step i's kernels overlap step i+1's "
                         "upload and step i-1's download (pinned host memory, own streams); "
                         "64 steps per captured CUDA graph")}
+    m.moe_check(path.ws)
 
     if rank != 0:
         if dist is not None:
@@ -711,17 +868,17 @@ def main():
     byts = algorithmic_bytes(w, kept_rows)
     peak, peak_kind = hbm_peak()
     kern = {}
-    for s, name in enumerate(probe_names):
+    for s, name in enumerate(path.probe_names):
         us = mean[s] * 1e3
         gbs = byts[name] / (mean[s] * 1e-3) / 1e9
         kern[name] = {"us": round(us, 2), "bytes": byts[name], "gbs": round(gbs, 1),
                       "frac": round(gbs / peak, 4)}
-    t_disp = mean[probe_names.index("dispatch")]
-    t_comb = mean[probe_names.index("combine")]
+    t_disp = mean[path.probe_names.index("dispatch")]
+    t_comb = mean[path.probe_names.index("combine")]
     dom = "dispatch" if t_disp >= t_comb else "combine"
     dom_gbs = byts[dom] / (max(t_disp, t_comb) * 1e-3) / 1e9
-    dc_ms = t_disp + t_comb
-    dc_gbs = (byts["dispatch"] + byts["combine"]) / (dc_ms * 1e-3) / 1e9
+    dc = dc_summary(w, kept_rows, t_disp, t_comb, peak)
+    dci = dc_summary(w, kept_rows, iso["dispatch"], iso["combine"], peak)
     ms_step = total_ms / K
     line = {
         "metric": METRIC,
@@ -736,25 +893,9 @@ def main():
         "vs_baseline": None,
         "dtype": "fp8-e4m3 dispatch, bf16 rows, fp32 accumulate" if w.fp8 else "bf16",
         "data": "synthetic",
-        "config": {"workload": w.describe(), "tokens": T, "hidden": w.H, "experts": w.E,
-                   "k": k, "ranks": w.R, "capacity": shape.capacity, "rows": N,
-                   "kept_rows": kept_rows, "parallelism": f"replicas x{world}",
-                   "l2": ("256 MiB write + read between timed steps, outside the step events"
-                          if flush_between else
-                          f"no flush: inputs larger than L2 ({touched / 1e6:.0f} MB touched per "
-                          f"step vs 126 MB L2), steps back to back"),
-                   "layout": ("per-source-rank: rows by destination rank, source shard "
-                              "(R shards of ceil(T/R) tokens), expert, token") if src else
-                             "rows by expert, token",
-                   "max_ranks": M if M > 0 else None,
-                   "bias_gamma": G if G > 0 else None,
-                   "router": args.router,
-                   "home_rank": HOME if HOME >= 0 else None,
-                   "step": " + ".join(names) + ", one CUDA graph"},
-        "dispatch_combine": {"tokens_per_s": world * T / (dc_ms * 1e-3),
-                             "us": round(dc_ms * 1e3, 2), "gbs": round(dc_gbs, 1),
-                             "frac": round(dc_gbs / peak, 4),
-                             "frac_of_8tbs": round(dc_gbs / 8000.0, 4),
+        "config": bench_config(w, args, world),
+        "kept_rows": kept_rows,
+        "dispatch_combine": {"tokens_per_s": world * T / ((t_disp + t_comb) * 1e-3), **dc,
                              "method": (f"in the step: a replay of the step with event records "
                                         f"between its kernels (no launch overlap across them), "
                                         f"mean of {K_ops}")},
@@ -765,35 +906,38 @@ def main():
             "method": ("torch device-to-device copy of the same bytes as dispatch + combine "
                        "(half read, half written), flushed L2, median")},
         "dispatch_combine_isolated": {
-            "tokens_per_s": world * T / ((iso["dispatch"] + iso["combine"]) * 1e-3),
-            "us": round((iso["dispatch"] + iso["combine"]) * 1e3, 2),
+            "tokens_per_s": world * T / ((iso["dispatch"] + iso["combine"]) * 1e-3), **dci,
             "dispatch_us": round(iso["dispatch"] * 1e3, 2),
             "combine_us": round(iso["combine"] * 1e3, 2),
-            "gbs": round((byts["dispatch"] + byts["combine"])
-                         / ((iso["dispatch"] + iso["combine"]) * 1e-3) / 1e9, 1),
-            "frac": round((byts["dispatch"] + byts["combine"])
-                          / ((iso["dispatch"] + iso["combine"]) * 1e-3) / 1e9 / peak, 4),
-            "frac_of_8tbs": round((byts["dispatch"] + byts["combine"])
-                                  / ((iso["dispatch"] + iso["combine"]) * 1e-3) / 1e9 / 8000.0,
-                                  4),
-            "method": (f"each op alone as a one-kernel CUDA graph, median of {iso_n}, "
+            "method": (f"each op alone as a one-kernel CUDA graph, median of {K_ops}, "
                        "256 MiB L2 write + read-back before each launch outside the events")},
         "kernels": kern,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(dom_gbs, 1),
                      "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
                      "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
                      "traffic": ncu_traffic(dom, w.name)},
-        "gpu_launches": kernels_per_step(args.path, separate, src,
-                                         small_route_layout(T, w.E, k), G > 0) * K,
+        "gpu_launches": kernels_per_step(args.path, path.separate, path.src,
+                                         small_route_layout(T, w.E, k),
+                                         args.bias_gamma > 0) * K,
         "clocks": clocks,
         "e2e": e2e,
     }
     if not args.no_cpu_baseline and world == 1:
-        v, tokens, reps, el = time_oracle(w, inp, args.cpu_seconds)
+        v, tokens, reps, el, stage_ms = time_oracle(w, path.inp, args.cpu_seconds)
         line["cpu_baseline"] = {
             "value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"{reps} single-threaded oracle passes over the first {tokens} of "
-                      f"{T} tokens of the same batch ({el:.1f} s)"}
+                      f"{T} tokens of the same batch ({el:.1f} s)",
+            **host_facts(), "stage_ms_per_pass": stage_ms}
+    del path, flush_buf
+    torch.cuda.empty_cache()
+    others = [n for n in args.per_workload.split(",") if n and n != "none" and n != w.name]
+    if world == 1 and others:
+        per = {}
+        for name in others:
+            per[name] = measure_workload(args, WORKLOADS[name], dev, stream, peak,
+                                         args.per_workload_steps, args.warmup)
+        line["per_workload"] = per
     print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()

@@ -62,7 +62,7 @@ def test_reference_arm_prints_one_line_and_other_ranks_stay_silent(capsys, monke
     import json
     import bench
     from combine_moe_route_07_b200.workloads import WORKLOADS
-    args = type("A", (), dict(gpus=2, steps=2, warmup=1))()
+    args = bench.parse(["--gpus", "2", "--steps", "2", "--warmup", "1"])
     monkeypatch.setenv("RANK", "1")
     assert bench.run_reference(args, WORKLOADS["tiny"]) == 0
     assert capsys.readouterr().out == ""
@@ -70,7 +70,10 @@ def test_reference_arm_prints_one_line_and_other_ranks_stay_silent(capsys, monke
     assert bench.run_reference(args, WORKLOADS["tiny"]) == 0
     line = json.loads(capsys.readouterr().out.strip())
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
-    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] == 1
+    assert cb["host_cores"] == os.cpu_count() and cb["usable_cores"] >= 1
+    assert "cpu_model" in cb and set(cb["stage_ms_per_step"]) == set(bench.STAGES)
     assert line["e2e"]["h2d_bytes_per_step"] == 0
     w = WORKLOADS["tiny"]
     cfg = line["config"]
@@ -78,6 +81,28 @@ def test_reference_arm_prints_one_line_and_other_ranks_stay_silent(capsys, monke
         (w.T, w.H, w.E, w.k, w.R)
     assert cfg["rows"] == w.rows and cfg["capacity"] == w.capacity
     assert line["metric"] == bench.METRIC and line["higher_is_better"] is True
+    # the kernel arm prints the same config object for the same arguments
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert cfg == bench.bench_config(w, args, 2)
+
+
+def test_step_plan_names_every_call_and_the_bias_update():
+    """The calls a step makes, for every bench variant; the bias update sits
+    before the combine whenever it is asked for."""
+    import bench
+    from combine_moe_route_07_b200.workloads import WORKLOADS
+    w = WORKLOADS["prefill"]
+    plan = lambda *a: bench.step_plan(w, bench.parse(list(a)))  # noqa: E731
+    assert plan() == (("route_layout_dispatch", "combine"), False)
+    assert plan("--path", "fused") == (("route_layout", "dispatch", "combine"), False)
+    assert plan("--path", "separate")[0] == ("route", "layout", "dispatch", "combine")
+    assert plan("--layout", "src") == (("route", "layout_src", "dispatch", "combine"), True)
+    assert plan("--max-ranks", "2")[0][0] == "route_limited"
+    assert plan("--router", "round_robin")[0][0] == "route_round_robin"
+    assert plan("--home", "3")[0][1] == "layout_remote_first"
+    for extra in ([], ["--path", "fused"], ["--path", "separate"], ["--layout", "src"]):
+        names = plan("--bias-gamma", "0.01", *extra)[0]
+        assert names[-2:] == ("bias_update", "combine")
 
 
 def test_algorithmic_bytes_cover_every_step_name():
