@@ -10,13 +10,17 @@
 // two tile tables) in a file-scope device array instead of a caller workspace.
 //
 // The array is kMoeNoallocScratchBytes bytes; every GPU that loads the library
-// holds it until the process exits.  The first call on a device looks up its
-// device address (cudaGetSymbolAddress, with that device current) and clears
-// it; make that first call before any stream capture.  Every call leaves the
-// array ready for the next one (the layout kernels clear the counters they
-// used); a call whose launch fails clears the whole array again.  Calls share
-// the array, so calls that overlap on the GPU (different streams, or different
-// host threads, without ordering) race and give wrong results.
+// holds it until the process exits.  Every call looks up the array's device
+// address on the current device (cudaGetSymbolAddress), so no address outlives
+// the context it came from (after cudaDeviceReset the library's module is
+// loaded again and its array has a new, zero-filled copy).  The first call that
+// sees an address on a device clears the array there; make that first call
+// before any stream capture.  Every call leaves the array ready for the next
+// one (the layout kernels clear the counters they used); a call whose launch
+// fails clears the whole array again.  Calls share the array, so calls that
+// overlap on the GPU (different streams, or different host threads, without
+// ordering) race and give wrong results.  The kernels' error word lives in the
+// array too; nothing reads it and nothing clears it (see the header).
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -34,25 +38,26 @@ constexpr size_t kMoeNoallocScratchBytes = kHeader + MOE_NOALLOC_TABLE_BYTES;
 static __device__ __align__(256) unsigned char g_layout_scratch[kMoeNoallocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_ptr[kMaxDevices] = {nullptr};
+void* g_cleared[kMaxDevices] = {nullptr};  // address last cleared on each device
 std::mutex g_scratch_mu;
 
-// Device address of the scratch array on the current device; the first call
-// per device resolves it and zero-fills the array.
+// Device address of the scratch array on the current device, looked up on
+// every call; the first call that sees an address on a device zero-fills the
+// array (cudaMemsetAsync on `stream`).
 moe_status_t scratch_for_current_device(cudaStream_t stream, void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_layout_scratch) != cudaSuccess || p == nullptr)
+    return MOE_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_layout_scratch) != cudaSuccess || p == nullptr)
-      return MOE_ERR_CUDA;
+  if (g_cleared[dev] != p) {
     if (cudaMemsetAsync(p, 0, kMoeNoallocScratchBytes, stream) != cudaSuccess)
       return MOE_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
+    g_cleared[dev] = p;
   }
-  *out = g_scratch_ptr[dev];
+  *out = p;
   return MOE_OK;
 }
 

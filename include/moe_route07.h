@@ -316,15 +316,19 @@ moe_status_t moe_combine(const moe_shape_t* shape, const void* y, const int32_t*
  * bytes, so min(ceil(T/16), 128) * E <= 65536 (any T for E <= 512, T <= 1024
  * for E = 1024); larger shapes return MOE_ERR_UNSUPPORTED and launch nothing.
  * Allocates nothing: no cudaMalloc / cudaFree or allocating library call.
- *  - The first call on a device resolves the array's device address and
- *    zero-fills it (cudaMemsetAsync on `stream`): make that first call before
- *    any stream capture.
+ *  - Every call looks up the array's device address on the current device
+ *    (cudaGetSymbolAddress), so an address never outlives its context (after
+ *    cudaDeviceReset the array is loaded again, zero-filled).  The first call
+ *    that sees an address on a device zero-fills the array there
+ *    (cudaMemsetAsync on `stream`): make that first call before any stream
+ *    capture.
  *  - Every call leaves the array ready for the next one; a call whose launch
  *    fails zero-fills it again.
  *  - All calls share the one array, so calls that overlap on the GPU race;
  *    order them (one stream, or events).
- *  - Device-side problems are not reported (there is no workspace to read
- *    them from); an id outside [0,E) still comes out as dst_pos -1. */
+ *  - Device-side problems are not reported: the kernels record the first one
+ *    in the array's error word, which no call reads or clears (an id outside
+ *    [0,E) still comes out as dst_pos -1). */
 #define MOE_NOALLOC_TABLE_BYTES (512u << 10)
 moe_status_t moe_layout_noalloc(const moe_shape_t* shape, const int32_t* ids, int32_t* counts,
                                 int32_t* expert_off, int32_t* rank_off, int32_t* rank_counts,

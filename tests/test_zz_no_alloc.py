@@ -4,8 +4,9 @@ runtimes whose pool owns the device, latency-critical code that may not call
 cudaMalloc).  Its scratch is a static device array inside the library.
 
 The GPU test calls it through the C ABI twice in a row on each shape and
-checks both results against the workspace-based moe_layout, bit for bit (the
-tolerance every layout test uses).  This file is collected last so that a run
+checks both results bit for bit (the tolerance every layout test uses)
+against the workspace-based moe_layout and against the oracle's layout of the
+same ids.  This file is collected last so that a run
 stopping at the first failure has run every other test already; it passes on
 its own in a fresh process as well.
 """
@@ -15,6 +16,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from combine_moe_route_07_b200 import _binding
 from combine_moe_route_07_b200.workloads import WORKLOADS, Workload, make_inputs
 
@@ -62,6 +64,7 @@ def test_noalloc_matches_workspace_layout_twice(w):
     ref = m.moe_layout(shape_py, ids, ws=ws)
     m.moe_check(ws)
     want = {f: getattr(ref, f).cpu().numpy() for f in FIELDS}
+    orc = oracle.layout(ids.cpu().numpy(), w.E, w.R, capacity=w.capacity, align=w.align)
 
     shape = _shape_c(w)
     for call in range(2):
@@ -74,7 +77,9 @@ def test_noalloc_matches_workspace_layout_twice(w):
         if call == 1:  # set-up is done; the call itself reserves no device memory
             assert torch.cuda.mem_get_info(dev)[0] == free_before
         for f in FIELDS:
-            assert np.array_equal(out[f].cpu().numpy(), want[f]), (call, f)
+            got = out[f].cpu().numpy()
+            assert np.array_equal(got, want[f]), (call, f)
+            assert np.array_equal(got, orc[f]), (call, f, "oracle")
 
 
 def test_noalloc_rejects_shapes_beyond_its_limit():
