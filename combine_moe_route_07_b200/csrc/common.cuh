@@ -28,10 +28,6 @@ __device__ __forceinline__ void report(WsHeader* h, int code, int detail) {
   if (atomicCAS(&h->err, 0, code) == 0) atomicExch(&h->detail, detail);
 }
 
-__device__ __forceinline__ int error_seen(const WsHeader* h) {
-  return *reinterpret_cast<const volatile int32_t*>(&h->err);
-}
-
 // Relaxed, GPU-scope 32-bit load/store (one word carries flag and value, so
 // no extra ordering is needed between them).
 __device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
