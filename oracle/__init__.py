@@ -56,6 +56,8 @@ def lib():
         L.orc_dispatch_fp8.restype = None
         L.orc_combine.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, i32]
         L.orc_combine.restype = None
+        L.orc_combine_f32.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, i32]
+        L.orc_combine_f32.restype = None
         L.orc_expert_scale.argtypes = [i32, i32, vp, vp, i32, vp, vp]
         L.orc_expert_scale.restype = None
         L.orc_dequant_fp8.argtypes = [i64, i32, vp, vp, vp]
@@ -236,8 +238,7 @@ def dispatch_fp8(x_bits, dst_pos, N):
     return out, scales
 
 
-def combine(y_bits, dst_pos, gates, T, shared_bits=None, residual_bits=None, tokens=None):
-    """uint16 [T,H] bf16 bits.  With `tokens`, only those rows are computed."""
+def _combine(fn, y_bits, dst_pos, gates, T, shared_bits, residual_bits, tokens):
     y_bits = _c(y_bits, np.uint16)
     dst_pos = _c(dst_pos, np.int32)
     gates = _c(gates, np.float32)
@@ -247,9 +248,23 @@ def combine(y_bits, dst_pos, gates, T, shared_bits=None, residual_bits=None, tok
     rs = None if residual_bits is None else _c(residual_bits, np.uint16)
     out = np.zeros((T, H), np.uint16)
     tk = None if tokens is None else _c(tokens, np.int32)
-    lib().orc_combine(T, H, k, _p(y_bits), _p(dst_pos), _p(gates), _p(sh), _p(rs), _p(out),
-                      _p(tk), 0 if tk is None else int(tk.shape[0]))
+    fn(T, H, k, _p(y_bits), _p(dst_pos), _p(gates), _p(sh), _p(rs), _p(out), _p(tk),
+       0 if tk is None else int(tk.shape[0]))
     return out
+
+
+def combine(y_bits, dst_pos, gates, T, shared_bits=None, residual_bits=None, tokens=None):
+    """The combine's exact sum (fp64), rounded once to bf16; uint16 [T,H]
+    bf16 bits.  With `tokens`, only those rows are computed."""
+    return _combine(lib().orc_combine, y_bits, dst_pos, gates, T, shared_bits, residual_bits,
+                    tokens)
+
+
+def combine_f32(y_bits, dst_pos, gates, T, shared_bits=None, residual_bits=None, tokens=None):
+    """The combine accumulated in binary32 in fixed order (slot fmaf's, then
+    shared, then residual), rounded once to bf16; arguments as combine()."""
+    return _combine(lib().orc_combine_f32, y_bits, dst_pos, gates, T, shared_bits,
+                    residual_bits, tokens)
 
 
 def expert_scale(xd_bits, expert_off, counts, capacity=0):

@@ -58,7 +58,10 @@
  * Precision: the pages fix none.  Decisions that turn floats into integers
  * (the top-k selection key, the e4m3 codes) are taken in fp32, the precision
  * the kernels decide in.  Everything else (gate softmax, combine sum) is
- * evaluated in fp64 and rounded once at the end.
+ * evaluated in fp64 and rounded once at the end.  The combine is also given
+ * in the accumulation the hot path is specified with (binary32, fixed slot
+ * order; orc_combine_f32), pinned against the fp64 sum by the binary32 error
+ * bound and by hand-worked cases where the order decides the result.
  *
  * Parity pins: every function here is pinned by CPU tests (brute force,
  * closed forms, library special cases, hand-worked fixtures); none is
@@ -682,6 +685,35 @@ void orc_combine(int T, int H, int k, const uint16_t* y, const int32_t* dst_pos,
       if (shared) acc += orc_bf16_to_double(shared[(size_t)t * H + c]);
       if (residual) acc += orc_bf16_to_double(residual[(size_t)t * H + c]);
       out[(size_t)t * H + c] = orc_double_to_bf16(acc);
+    }
+  }
+}
+
+/* The same sum accumulated in binary32 in a fixed order: acc = +0; for each
+ * kept slot j = 0..k-1, acc = fmaf(gates[t,j], y[dst_pos[t,j], c], acc) (one
+ * fused multiply-add, one rounding); then acc = acc + shared[t,c]; then acc =
+ * acc + residual[t,c] (one binary32 addition each); out = bf16 of acc, nearest
+ * even.  Each step rounds once to binary32 (unit roundoff 2^-24), so with n
+ * steps |acc - exact sum| <= n * 2^-24 * (1+2^-24)^n * (sum of the terms'
+ * magnitudes); that difference decides the bf16 rounding where the exact sum
+ * lies at or next to a bf16 midpoint, and dominates where the terms cancel.
+ * Arguments as orc_combine. */
+void orc_combine_f32(int T, int H, int k, const uint16_t* y, const int32_t* dst_pos,
+                     const float* gates, const uint16_t* shared, const uint16_t* residual,
+                     uint16_t* out, const int32_t* tokens, int n_tokens) {
+  int n = tokens ? n_tokens : T;
+  for (int i = 0; i < n; ++i) {
+    int t = tokens ? tokens[i] : i;
+    for (int c = 0; c < H; ++c) {
+      float acc = 0.0f;
+      for (int j = 0; j < k; ++j) {
+        int32_t p = dst_pos[(size_t)t * k + j];
+        if (p < 0) continue;
+        acc = fmaf(gates[(size_t)t * k + j], bf16_to_float(y[(size_t)p * H + c]), acc);
+      }
+      if (shared) acc = acc + bf16_to_float(shared[(size_t)t * H + c]);
+      if (residual) acc = acc + bf16_to_float(residual[(size_t)t * H + c]);
+      out[(size_t)t * H + c] = float_to_bf16(acc);
     }
   }
 }

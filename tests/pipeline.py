@@ -133,9 +133,29 @@ def run_oracle(w: Workload, inp, through="combine"):
     y = standin_oracle(w, disp, L)
     res["y"] = y
     res["shared"] = bf16_bits(inp.shared) if w.shared else None
-    res["out"] = oracle.combine(y, L["dst_pos"], gates, w.T, shared_bits=res["shared"],
-                                residual_bits=x if w.residual else None)
+    res.update(oracle_combines(y, L["dst_pos"], gates, w.T, res["shared"],
+                               x if w.residual else None))
     return res
+
+
+def _abs_bits(b):
+    return None if b is None else (np.asarray(b) & 0x7FFF).astype(np.uint16)
+
+
+def oracle_combines(y, dst_pos, gates, T, shared_bits=None, residual_bits=None):
+    """The oracle's combine three ways: `out` the exact sum rounded once to
+    bf16; `out_f32` the fixed-order binary32 accumulation (slot fmaf's, then
+    shared, then residual) rounded once; `mag` the bf16 of the sum of the
+    terms' magnitudes (for the binary32 error bound)."""
+    return {
+        "out": oracle.combine(y, dst_pos, gates, T, shared_bits=shared_bits,
+                              residual_bits=residual_bits),
+        "out_f32": oracle.combine_f32(y, dst_pos, gates, T, shared_bits=shared_bits,
+                                      residual_bits=residual_bits),
+        "mag": oracle.combine(_abs_bits(y), dst_pos, np.abs(gates), T,
+                              shared_bits=_abs_bits(shared_bits),
+                              residual_bits=_abs_bits(residual_bits)),
+    }
 
 
 def oracle_chunk(w: Workload, x_bits, ids, gates, dst_pos, tokens, shared_bits=None):
@@ -165,14 +185,9 @@ def oracle_chunk(w: Workload, x_bits, ids, gates, dst_pos, tokens, shared_bits=N
     if w.shared:
         assert shared_bits is not None, "the workload has a shared expert: pass its output"
         sh = shared_bits[tokens]
-    out = oracle.combine(y, local, gates[tokens], n, shared_bits=sh,
-                         residual_bits=xs if w.residual else None)
-    return {"keep": keep, "dispatch": disp, "out": out}
-
-
-def oracle_combine_sampled(w: Workload, x_bits, ids, gates, dst_pos, tokens, shared_bits=None):
-    """Oracle combine for a sample of tokens (see oracle_chunk)."""
-    return oracle_chunk(w, x_bits, ids, gates, dst_pos, tokens, shared_bits)["out"]
+    res = {"keep": keep, "dispatch": disp}
+    res.update(oracle_combines(y, local, gates[tokens], n, sh, xs if w.residual else None))
+    return res
 
 
 def _scale_rows(w, y, e_of_row):
@@ -214,6 +229,52 @@ def assert_bf16_close(got_bits, want_bits, ulps=1, what=""):
     assert bad == 0, f"{what}: {bad} of {d.size} values differ by more than {ulps} bf16 ulp " \
                      f"(max {int(d.max())})"
     return d
+
+
+def bf16_value(bits):
+    """bf16 bit patterns -> float64 values."""
+    return (np.asarray(bits).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def bf16_quantum(v):
+    """Spacing of the bf16 numbers at |v| (2^-133 at zero and below the
+    normal range)."""
+    a = np.abs(v)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, 2.0 ** (np.maximum(e, -126) - 7), 2.0 ** -133)
+
+
+def assert_combine(got_bits, want, k, what, exact_rows=None):
+    """The combine tolerance, derived from the arithmetic.  The kernels
+    accumulate in binary32 in fixed order (slot FMAs, then shared, then
+    residual) and round once to bf16, so they must equal the oracle's
+    fixed-order accumulation `out_f32` bit for bit (+0 and -0 alike) on the
+    rows in `exact_rows` (all rows by default; the whole-path tests leave out
+    tokens whose gates came out one fp32 ulp away from the oracle's).  Every
+    value must also lie within one bf16 quantum plus the binary32 bound
+    (k+2) * 2^-24 * (sum of the terms' magnitudes) of the exact sum `out`: one
+    bf16 ulp wherever the terms do not cancel.  Returns the ulp distance to
+    the exact sum."""
+    got_bits = np.asarray(got_bits)
+    d32 = bf16_ulp_diff(got_bits, want["out_f32"])
+    sel = d32 if exact_rows is None else d32[exact_rows]
+    bad = int((sel != 0).sum())
+    assert bad == 0, f"{what}: {bad} of {sel.size} values differ from the fixed-order binary32 " \
+                     f"accumulation (max {int(sel.max())} ulp)"
+    g = bf16_value(got_bits)
+    e = bf16_value(want["out"])
+    mag = bf16_value(want["mag"]) * (1 + 2.0 ** -7)
+    allow = np.maximum(bf16_quantum(g), bf16_quantum(e)) + (k + 2) * 2.0 ** -24 * mag * (1 + 1e-6)
+    over = int((np.abs(g - e) > allow).sum())
+    assert over == 0, f"{what}: {over} values outside the binary32 bound of the exact sum"
+    return bf16_ulp_diff(got_bits, want["out"])
+
+
+def gate_rows_equal(gpu_gates, oracle_gates):
+    """Tokens whose gates are bit-identical on both sides."""
+    a = np.ascontiguousarray(gpu_gates, np.float32).view(np.uint32)
+    b = np.ascontiguousarray(oracle_gates, np.float32).view(np.uint32)
+    return (a == b).all(axis=1)
 
 
 def assert_gates_close(got, want, rel=1e-6, what="gates"):

@@ -22,6 +22,8 @@ void orc_dispatch_bf16(int, int, int, const uint16_t*, const int32_t*, uint16_t*
 void orc_dispatch_fp8(int, int, int, const uint16_t*, const int32_t*, uint8_t*, float*);
 void orc_combine(int, int, int, const uint16_t*, const int32_t*, const float*, const uint16_t*,
                  const uint16_t*, uint16_t*, const int32_t*, int);
+void orc_combine_f32(int, int, int, const uint16_t*, const int32_t*, const float*, const uint16_t*,
+                 const uint16_t*, uint16_t*, const int32_t*, int);
 void orc_dequant_fp8(int64_t, int, const uint8_t*, const float*, uint16_t*);
 uint8_t orc_e4m3_encode_satfinite(float);
 double orc_e4m3_decode(uint8_t);
@@ -71,6 +73,8 @@ static int run(int T, int E, int k, int R, int C, int align, int H) {
   int32_t tok[2] = {0, T - 1};
   orc_combine(T, H, k, xd, dst, gates, x, x, out, NULL, 0);
   orc_combine(T, H, k, xd, dst, gates, NULL, NULL, out, tok, T > 0 ? 2 : 0);
+  orc_combine_f32(T, H, k, xd, dst, gates, x, x, out, NULL, 0);
+  orc_combine_f32(T, H, k, xd, dst, gates, NULL, NULL, out, tok, T > 0 ? 2 : 0);
   if (H % 128 == 0) {
     uint8_t* q = xmalloc((N ? N : 1) * H);
     float* s = xmalloc(4 * (N ? N : 1) * (H / 128));

@@ -23,15 +23,19 @@ an operand read twice, dropped, or taken from the wrong token or slice.
 `test_inputs_tell_the_operands_apart` shows, on the CPU, that each of those
 mistakes moves most outputs by more than the 1-ulp tolerance.
 
-Tolerance (as in every combine test): 1 bf16 ulp against the oracle's fp64
-sum, and >= 99.9 % of the values exact.
+Tolerance (as in every combine test, pipeline.assert_combine): bit for bit
+against the oracle's fixed-order binary32 accumulation, and within one bf16
+quantum plus the binary32 error bound of the exact sum.  With a shared row
+and a residual that are independent draws, the sum sometimes nearly cancels;
+there the bound, not one ulp, is what any binary32 accumulation can promise.
 """
 import numpy as np
 import pytest
 import torch
 
 from combine_moe_route_07_b200.workloads import WORKLOADS, Workload, make_inputs
-from pipeline import (assert_bf16_close, bf16_ulp_diff, run_gpu, run_oracle, shape_of, to_np)
+from pipeline import (assert_combine, bf16_ulp_diff, gate_rows_equal, run_gpu, run_oracle,
+                      shape_of, to_np)
 
 BOTH = dict(shared=True, residual=True)
 CASES = [
@@ -66,8 +70,9 @@ def test_whole_path_with_distinct_shared_and_residual(w, fused):
     o = run_oracle(w, inp)
     g = run_gpu(w, inp, fused=fused)
     assert m.moe_get_device_error(g["ws"]) == (0, 0)
-    d = assert_bf16_close(to_np(g["out"]), o["out"], 1, w.name)
-    assert (d == 0).mean() > 0.999
+    d = assert_combine(to_np(g["out"]), o, w.k, w.name,
+                       exact_rows=gate_rows_equal(to_np(g["gates"]), o["gates"]))
+    assert (d <= 1).mean() > 0.999
 
 
 @pytest.mark.gpu
@@ -88,8 +93,8 @@ def test_combine_on_oracle_operands(w):
     out = m.moe_combine(shape, y, dst, gates, ws=ws, shared=sh, residual=rs)
     torch.cuda.synchronize()
     assert m.moe_get_device_error(ws) == (0, 0)
-    d = assert_bf16_close(to_np(out), o["out"], 1, w.name)
-    assert (d == 0).mean() > 0.999
+    d = assert_combine(to_np(out), o, w.k, w.name)
+    assert (d <= 1).mean() > 0.999
 
 
 def test_inputs_tell_the_operands_apart():

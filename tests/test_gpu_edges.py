@@ -8,8 +8,8 @@ import pytest
 import torch
 
 from combine_moe_route_07_b200.workloads import Workload, make_inputs
-from pipeline import (assert_bf16_close, assert_gates_close, run_gpu, run_oracle, shape_of,
-                      to_np)
+from pipeline import (assert_combine, assert_gates_close, gate_rows_equal, run_gpu, run_oracle,
+                      shape_of, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -34,7 +34,8 @@ def _check_all(w, inp=None, fused=False):
         assert np.array_equal(to_np(s)[used], o["dispatch"][1][used])
     else:
         assert np.array_equal(to_np(g["dispatch"])[used], o["dispatch"][used])
-    assert_bf16_close(to_np(g["out"]), o["out"], 1, w.name)
+    assert_combine(to_np(g["out"]), o, w.k, w.name,
+                   exact_rows=gate_rows_equal(to_np(g["gates"]), o["gates"]))
 
 
 CASES = [

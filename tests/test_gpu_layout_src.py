@@ -9,7 +9,7 @@ import torch
 
 import oracle
 from combine_moe_route_07_b200.workloads import WORKLOADS, Workload, bf16_bits, make_inputs
-from pipeline import assert_bf16_close, to_np
+from pipeline import _scale_rows, assert_combine, gate_rows_equal, oracle_combines, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -160,14 +160,21 @@ def test_dispatch_and_combine_over_the_src_layout(capacity_factor):
     torch.cuda.synchronize()
     assert m.moe_get_device_error(ws) == (0, 0)
 
-    o = oracle.layout_src(ids_np, w.E, w.R, capacity=C)
+    # the oracle's own path: route, per-source-rank layout, dispatch
+    o_ids, o_gates = oracle.route(inp.logits.numpy(), w.k, renorm=w.renorm)
+    assert np.array_equal(o_ids, ids_np)
+    o = oracle.layout_src(o_ids, w.E, w.R, capacity=C)
     _compare(lay, o, "path")
     xb = bf16_bits(inp.x)
     rows = oracle.dispatch_bf16(xb, o["dst_pos"], shape.rows)
     used = o["src_idx"] >= 0
     assert np.array_equal(to_np(xd).view(np.uint16)[used], rows[used])
-    # the combine over the same expert rows the GPU combined (the stand-in
-    # expert is outside the path)
-    want = oracle.combine(to_np(y), o["dst_pos"], to_np(gates), w.T,
-                          shared_bits=bf16_bits(inp.shared), residual_bits=xb)
-    assert_bf16_close(to_np(out), want, 1, "src_path")
+    # the oracle's combine over its own expert rows: the same stand-in expert
+    # (row of expert e times (e+1)/E) applied to the oracle's dispatch
+    o_src = o["src_idx"]
+    o_e = np.where(o_src >= 0, o_ids.ravel()[np.maximum(o_src, 0)], 0).astype(np.int32)
+    o_y = _scale_rows(w, rows, o_e)
+    want = oracle_combines(o_y, o["dst_pos"], o_gates, w.T,
+                           shared_bits=bf16_bits(inp.shared), residual_bits=xb)
+    assert_combine(to_np(out), want, w.k, "src_path",
+                   exact_rows=gate_rows_equal(to_np(gates), o_gates))

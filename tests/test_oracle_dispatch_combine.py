@@ -207,3 +207,109 @@ def test_hand_worked_combine():
         out = _bits_to_f64(oracle.combine(y, L["dst_pos"], gates, 2))
         assert out[0].tolist() == [float(v) for v in g[f"out_{tag}_t0"]]
         assert out[1].tolist() == [float(v) for v in g[f"out_{tag}_t1"]]
+
+
+# ---- the combine in fixed-order binary32 accumulation (orc_combine_f32) ----
+
+def _one_token_case(g, tag):
+    vals = lambda key: [float(v) for v in g[key]]  # noqa: E731
+    gates = np.array([vals(f"{tag}_gates")], np.float32)
+    y = bf16_bits(torch.tensor(vals(f"{tag}_y"))[:, None].to(torch.bfloat16))
+    dst = np.array([[int(v) for v in g[f"{tag}_dst"]]], np.int32)
+    extra = {}
+    for key in ("shared", "residual"):
+        if f"{tag}_{key}" in g:
+            extra[f"{key}_bits"] = bf16_bits(torch.tensor([vals(f"{tag}_{key}")]).to(torch.bfloat16))
+    return y, dst, gates, extra
+
+
+@pytest.mark.parametrize("tag", ["c1", "c2", "c3", "c4", "c5"])
+def test_hand_worked_combine_accumulation_order(tag):
+    """Hand-worked cases where the binary32 order decides the result (a tie
+    at 2^24 lost in one slot order and kept in another; shared before
+    residual; one rounding per fused multiply-add; a dropped slot)."""
+    g = read_golden("hand_combine_f32.txt")
+    y, dst, gates, extra = _one_token_case(g, tag)
+    f32 = _bits_to_f64(oracle.combine_f32(y, dst, gates, 1, **extra))[0, 0]
+    exact = _bits_to_f64(oracle.combine(y, dst, gates, 1, **extra))[0, 0]
+    assert f32 == float(g[f"{tag}_f32"][0])
+    assert exact == float(g[f"{tag}_exact"][0])
+
+
+def test_combine_f32_equals_exact_sum_when_every_step_is_exact():
+    """Gates that are powers of two and small integer rows keep every binary32
+    partial sum exact, so the fixed-order accumulation is the exact sum."""
+    rng = np.random.default_rng(31)
+    T, H, E, R, k = 64, 32, 16, 4, 6
+    x = bf16_bits(torch.from_numpy(rng.integers(-64, 65, (T, H)).astype(np.float32))
+                  .to(torch.bfloat16))
+    sh = bf16_bits(torch.from_numpy(rng.integers(-64, 65, (T, H)).astype(np.float32))
+                   .to(torch.bfloat16))
+    y = bf16_bits(torch.from_numpy(rng.integers(-64, 65, (T * k, H)).astype(np.float32))
+                  .to(torch.bfloat16))
+    gates = (2.0 ** -rng.integers(0, 4, (T, k))).astype(np.float32)
+    L = oracle.layout(_ids(T, E, k, rng), E, R)
+    for extra in ({}, {"shared_bits": sh}, {"residual_bits": x},
+                  {"shared_bits": sh, "residual_bits": x}):
+        a = oracle.combine_f32(y, L["dst_pos"], gates, T, **extra)
+        b = oracle.combine(y, L["dst_pos"], gates, T, **extra)
+        assert np.array_equal(a, b)
+
+
+def _bf16_quantum(v):
+    a = np.abs(v)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, 2.0 ** (np.maximum(e, -126) - 7), 2.0 ** -133)
+
+
+@pytest.mark.parametrize("case", ["random", "identity_experts", "cancelling"])
+def test_combine_f32_within_the_binary32_bound_of_the_exact_sum(case):
+    """|out - exact| <= half a bf16 quantum of out + n * 2^-24 * (sum of the
+    terms' magnitudes) * (1 + 1e-6), n = roundings (kept slots + shared +
+    residual): the standard bound for n binary32 steps.  A dropped term, a
+    wrong sign or a wrong row breaks it by orders of magnitude."""
+    rng = np.random.default_rng({"random": 41, "identity_experts": 42, "cancelling": 43}[case])
+    T, H, E, R, k = 300, 64, 32, 4, 8
+    x = _bf16_rand((T, H), rng)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    ids, gates = oracle.route(logits, k)
+    L = oracle.layout(ids, E, R)
+    if case == "identity_experts":
+        y = oracle.dispatch_bf16(x, L["dst_pos"], T * k)
+        sh = _bf16_rand((T, H), rng)
+    elif case == "cancelling":
+        y = oracle.dispatch_bf16(x, L["dst_pos"], T * k)
+        # shared = -(2x) up to bf16 rounding: the sum nearly cancels
+        sh = bf16_bits((-2.0 * bits_to_bf16(x).to(torch.float32)
+                        + torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)) * 1e-3)
+                       .to(torch.bfloat16))
+    else:
+        y = _bf16_rand((T * k, H), rng)
+        sh = _bf16_rand((T, H), rng)
+    out = _bits_to_f64(oracle.combine_f32(y, L["dst_pos"], gates, T, shared_bits=sh,
+                                          residual_bits=x))
+    yf = _bits_to_f64(y)[L["dst_pos"]]                # [T,k,H]
+    terms = gates.astype(np.float64)[:, :, None] * yf  # exact products
+    exact = terms.sum(1) + _bits_to_f64(sh) + _bits_to_f64(x)
+    mag = np.abs(terms).sum(1) + np.abs(_bits_to_f64(sh)) + np.abs(_bits_to_f64(x))
+    n = k + 2
+    allow = 0.5 * _bf16_quantum(out) + n * 2.0 ** -24 * mag * (1 + 1e-6)
+    assert np.all(np.abs(out - exact) <= allow)
+    # and the bound has teeth: against the exact sum with slot 0 left out, or
+    # with the residual counted twice, most values break it
+    assert (np.abs(out - (exact - terms[:, 0])) > allow).mean() > 0.9
+    assert (np.abs(out - (exact + _bits_to_f64(x))) > allow).mean() > 0.9
+
+
+def test_combine_f32_identity_experts_return_the_input_exactly():
+    """Identity experts with renormalised gates return x, also in the
+    fixed-order binary32 accumulation (the gates' sum is 1 to within a few
+    2^-24, far inside half a bf16 quantum)."""
+    rng = np.random.default_rng(44)
+    T, H, E, R, k = 200, 32, 64, 8, 10
+    x = _bf16_rand((T, H), rng)
+    ids, gates = oracle.route(rng.standard_normal((T, E)).astype(np.float32), k)
+    L = oracle.layout(ids, E, R)
+    y = oracle.dispatch_bf16(x, L["dst_pos"], T * k)
+    out = oracle.combine_f32(y, L["dst_pos"], gates, T)
+    assert np.array_equal(_bits_to_f64(out), _bits_to_f64(x))
