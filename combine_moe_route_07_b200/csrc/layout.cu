@@ -30,6 +30,7 @@
 // pass reads the table its count pass filled and clears the other one (the
 // rows the previous call left), so no clearing sits on the critical path.
 // Integer adds make every result independent of the order the CTAs run in.
+#include "block_scan.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -93,47 +94,6 @@ struct PlaceParams {
   int32_t* dst_pos;
   int32_t* src_idx;
 };
-
-// Exclusive scan of v[0..n) in shared memory by the whole CTA (n <= 4 *
-// THREADS).  Returns the total to every thread.
-template <int THREADS>
-__device__ int block_exclusive_scan(int32_t* v, int n, int32_t* warp_tot) {
-  constexpr int kW = THREADS / 32;
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int per = (n + THREADS - 1) / THREADS;
-  const int lo = threadIdx.x * per;
-  int local = 0;
-  for (int i = 0; i < per; ++i)
-    if (lo + i < n) local += v[lo + i];
-  int x = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(kFull, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) warp_tot[wid] = x;
-  __syncthreads();
-  if (wid == 0) {
-    int s = (lane < kW) ? warp_tot[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(kFull, s, o);
-      if (lane >= o) s += y;
-    }
-    if (lane < kW) warp_tot[lane] = s;
-  }
-  __syncthreads();
-  int run = (wid > 0 ? warp_tot[wid - 1] : 0) + x - local;
-  const int total = warp_tot[kW - 1];
-  for (int i = 0; i < per; ++i)
-    if (lo + i < n) {
-      const int t = v[lo + i];
-      v[lo + i] = run;
-      run += t;
-    }
-  __syncthreads();
-  return total;
-}
 
 constexpr size_t place_smem_words(int E, int staged_entries) {
   return (size_t)(kPlaceThreads / 32) * E + 5 * (size_t)E + 2 + 2 * (size_t)staged_entries;
