@@ -18,7 +18,9 @@
 // lane issues the 16-byte loads of up to KB slots before using any of them.
 // Bulk variant (dense layouts with many row slices per warp): the row slices
 // arrive in shared memory by bulk copy (TMA), several tokens ahead of the
-// arithmetic, so the bytes in flight do not cost registers.
+// arithmetic, so the bytes in flight do not cost registers.  Staged variant
+// (dense layouts with rows wider than 8 KiB): one ring per CTA, a producer
+// warp bringing in slices of several KiB per slot, eight consumer warps.
 #include <cuda_bf16.h>
 
 #include "bulk.cuh"
@@ -360,6 +362,174 @@ __global__ void __launch_bounds__(kBulkMaxWarps * 32, 1)
   }
 }
 
+// Staged variant: one ring of shared-memory stages per CTA, filled by one
+// producer warp and read by kStageConsumers consumer warps.  A unit is a slice
+// of SL bytes (a whole row, or an even part of it) of one token; its stage
+// holds that slice of each kept slot's y row, then of the shared-expert row,
+// then of the residual row, each brought in by ONE bulk copy of SL bytes
+// (lane j of the producer copies slot j) -- bulk copies of a few KiB reach the
+// DRAM read rate where 512-byte copies are bound by the copies' own cost.  The
+// producer also leaves the unit's gates, kept-slot mask, token and slice in the
+// stage's metadata before it arrives on the stage's "full" barrier; the
+// consumer warps split the slice's 16-byte chunks, accumulate each in fp32 in
+// slot order (fma.rn.f32x2), add the shared and residual rows, store the bf16
+// result, and arrive on the stage's "empty" barrier.  Each CTA takes a
+// contiguous range of units.  Every wait is bounded: a wait that gives up sets
+// MOE_ERR_DEVICE_TIMEOUT and the abort flag, the producer stops issuing, and
+// before it returns waits (bounded) for the copies of its last `ns` units, the
+// only ones whose landing it has not already seen.
+constexpr int kStageConsumers = 8;
+constexpr int kStageThreads = (kStageConsumers + 1) * 32;
+constexpr int kStageMax = 16;
+constexpr int kStageMinRing = 3;    // stages the slice width is chosen for
+constexpr size_t kStageSmemBudget = 200u * 1024u;
+
+struct StageMeta {
+  float gate[16];
+  uint32_t kept;
+  int token;
+  uint32_t off;  // byte offset of the slice in the row
+  uint32_t len;  // bytes of the slice
+};
+
+template <int KMAX>
+__global__ void __launch_bounds__(kStageThreads, 1)
+    combine_stage_kernel(const char* __restrict__ y, const int32_t* __restrict__ dst_pos,
+                         const float* __restrict__ gates, const char* __restrict__ shared,
+                         const char* __restrict__ residual, int T, int H, int k, int64_t N,
+                         char* __restrict__ out, WsHeader* hdr, int ns, uint32_t SL, int nsl) {
+  extern __shared__ __align__(128) unsigned char sbuf[];
+  __shared__ uint64_t full[kStageMax], empty[kStageMax];
+  __shared__ StageMeta meta[kStageMax];
+  __shared__ volatile int abort_flag;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int extra = (shared != nullptr) + (residual != nullptr);
+  const uint32_t row = (uint32_t)H * 2;
+  const size_t stage_bytes = (size_t)(k + extra) * SL;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ns; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kStageConsumers);
+    }
+    abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  pdl_wait();  // y, gates and dst_pos may come from the kernel launched just before
+  pdl_trigger();
+  const int64_t units = (int64_t)T * nsl;
+  const int64_t u0 = units * blockIdx.x / gridDim.x, u1 = units * (blockIdx.x + 1) / gridDim.x;
+  const int n = (int)(u1 - u0);
+
+  if (w == kStageConsumers) {  // the producer warp
+    // slot `lane` of the current token (p, g) and of the next one (np, ng),
+    // fetched one token ahead so their latency overlaps this token's copies
+    auto fetch = [&](int t, int& pp, float& gg) {
+      pp = -1;
+      gg = 0.0f;
+      if (t < T && lane < k) {
+        pp = __ldg(dst_pos + (size_t)t * k + lane);
+        gg = __ldg(gates + (size_t)t * k + lane);
+      }
+    };
+    int cur_t = n > 0 ? (int)(u0 / nsl) : 0, p, np;
+    float g, ng;
+    fetch(cur_t, p, g);
+    fetch(cur_t + 1, np, ng);
+    if (p >= N) {
+      report(hdr, MOE_ERR_DEVICE_RANGE, p);
+      p = -1;
+    }
+    int issued = 0;
+    for (int i = 0; i < n; ++i) {
+      const int s = i % ns;
+      if (i >= ns) {  // the consumers have finished with this stage's previous unit
+        const bool ok = __all_sync(
+            kFull, mbar_wait_bounded(&empty[s], (uint32_t)((i / ns) - 1) & 1u, kBulkTimeoutNs));
+        if (!ok) {
+          if (lane == 0) report(hdr, MOE_ERR_DEVICE_TIMEOUT, (int)(u0 + i));
+          abort_flag = 1;
+        }
+      }
+      if (__any_sync(kFull, abort_flag != 0)) break;  // one decision for the warp
+      const int64_t u = u0 + i;
+      const int t = (int)(u / nsl), sl = (int)(u - (int64_t)t * nsl);
+      if (t != cur_t) {  // units are consecutive: t == cur_t + 1
+        cur_t = t;
+        p = np;
+        g = ng;
+        if (p >= N) {
+          report(hdr, MOE_ERR_DEVICE_RANGE, p);
+          p = -1;
+        }
+        fetch(t + 1, np, ng);
+      }
+      const uint32_t off = (uint32_t)sl * SL;
+      const uint32_t len = min(SL, row - off);
+      const unsigned kept = __ballot_sync(kFull, p >= 0);
+      if (lane < KMAX) meta[s].gate[lane] = g;
+      if (lane == 0) {
+        meta[s].kept = kept;
+        meta[s].token = t;
+        meta[s].off = off;
+        meta[s].len = len;
+      }
+      __syncwarp();
+      if (lane == 0)  // after the metadata: the arrival releases it to the consumers
+        mbar_arrive_expect_tx(&full[s], ((uint32_t)__popc(kept) + (uint32_t)extra) * len);
+      __syncwarp();
+      unsigned char* sp = sbuf + (size_t)s * stage_bytes;
+      if (p >= 0) bulk_load(sp + (size_t)lane * SL, y + (size_t)p * row + off, len, &full[s]);
+      if (lane == 0 && shared != nullptr)
+        bulk_load(sp + (size_t)k * SL, shared + (size_t)t * row + off, len, &full[s]);
+      if (lane == 1 && residual != nullptr)
+        bulk_load(sp + (size_t)(k + extra - 1) * SL, residual + (size_t)t * row + off, len,
+                  &full[s]);
+      issued = i + 1;
+    }
+    if (lane == 0 && abort_flag) {  // the copies of the last ns units land before the CTA exits
+      for (int i = issued > ns ? issued - ns : 0; i < issued; ++i)
+        (void)mbar_wait_bounded(&full[i % ns], (uint32_t)(i / ns) & 1u, kBulkTimeoutNs);
+    }
+    return;
+  }
+
+  // the consumer warps: chunk c = (w*32 + lane) + kStageConsumers*32*r of the slice
+  for (int i = 0; i < n; ++i) {
+    const int s = i % ns;
+    const bool ok =
+        __all_sync(kFull, mbar_wait_bounded(&full[s], (uint32_t)(i / ns) & 1u, kBulkTimeoutNs));
+    if (!ok) {
+      if (lane == 0) report(hdr, MOE_ERR_DEVICE_TIMEOUT, (int)(u0 + i));
+      abort_flag = 1;
+    }
+    if (__any_sync(kFull, abort_flag != 0)) return;  // one decision for the warp
+    const StageMeta& m = meta[s];
+    const unsigned kept = m.kept;
+    const uint32_t len = m.len;
+    const unsigned char* sp = sbuf + (size_t)s * stage_bytes;
+    char* orow = out + (size_t)m.token * row + m.off;
+    for (uint32_t c = (uint32_t)(w * 32 + lane) * 16; c < len; c += kStageConsumers * 32 * 16) {
+      float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (j < k && ((kept >> j) & 1u))
+          fma8_x2(acc, m.gate[j], *reinterpret_cast<const uint4*>(sp + (size_t)j * SL + c));
+      if (shared != nullptr) add8(acc, *reinterpret_cast<const uint4*>(sp + (size_t)k * SL + c));
+      if (residual != nullptr)
+        add8(acc, *reinterpret_cast<const uint4*>(sp + (size_t)(k + extra - 1) * SL + c));
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      st16(orow + c, o);
+    }
+    __syncwarp();  // every lane is done with the stage
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+}
+
 // Enough CTAs for one warp per task, at most the ones resident at once.
 template <typename K>
 int grid_for(K kernel, const LaunchEnv& env, int64_t tasks) {
@@ -383,12 +553,40 @@ cudaError_t launch_combine(const LaunchEnv& env, const void* y, const int32_t* d
   const char* sh = static_cast<const char*>(shared);
   const char* rs = static_cast<const char*>(residual);
   char* o = static_cast<char*>(out);
+  const int extra = (shared != nullptr) + (residual != nullptr);
+  // Dense layouts with rows wider than 8 KiB and at least 8 units per SM: the
+  // staged variant, slices as wide as a ring of kStageMinRing stages allows
+  // (whole rows, or the row cut evenly into 16-byte multiples).  On 14 KiB
+  // rows its 7 KiB copies beat the bulk variant's 512-byte ones (Skewed
+  // dropless combine 711 -> 650 us); on 8 KiB rows and narrower (Prefill,
+  // Fine-grained) the bulk variant's 24 independent rings per SM do better.
+  if ((size_t)H * 2 > 8192) {
+    const size_t slots = (size_t)(k + extra);
+    const size_t row = (size_t)H * 2;
+    int64_t nsl = (int64_t)((slots * row * kStageMinRing + kStageSmemBudget - 1) / kStageSmemBudget);
+    if (nsl < 1) nsl = 1;
+    const uint32_t SL = (uint32_t)(((row + nsl - 1) / nsl + 15) / 16 * 16);
+    nsl = (int64_t)((row + SL - 1) / SL);
+    int ns = (int)(kStageSmemBudget / (slots * SL));
+    if (ns > kStageMax) ns = kStageMax;
+    if (!sparse && k <= 16 && ns >= 2 && (int64_t)T * nsl >= 8 * (int64_t)env.num_sms) {
+      const size_t smem = (size_t)ns * slots * SL;
+      auto kern = k <= 8 ? combine_stage_kernel<8> : combine_stage_kernel<16>;
+      int per_sm = 1;
+      const cudaError_t err =
+          blocks_per_sm(reinterpret_cast<const void*>(kern), kStageThreads, smem, &per_sm);
+      if (err != cudaSuccess) return err;
+      int64_t grid = (int64_t)env.num_sms * per_sm;
+      if (grid > (int64_t)T * nsl) grid = (int64_t)T * nsl;
+      return launch_pdl(env, kern, dim3((unsigned)grid), dim3(kStageThreads), smem, ys, dst_pos,
+                        gates, sh, rs, T, H, k, N, o, hdr, ns, SL, (int)nsl);
+    }
+  }
   // Dense layouts with at least 8 row slices per warp of a full bulk grid:
   // the bulk variant, when the stages of up to 12 slots (k plus the shared
   // and residual rows) fit twice per warp.  Warps matter more than ring
   // depth: 24 warps with two stages each tie or beat 16 with three, and wider
   // slices with fewer warps ran far slower.
-  const int extra = (shared != nullptr) + (residual != nullptr);
   const uint32_t stage_bytes = (uint32_t)(k + extra) * kBulkSlice;
   const int W = kBulkSmemBudget / ((size_t)kBulkMaxWarps * stage_bytes) >= 2 ? kBulkMaxWarps
                                                                              : kBulkMinWarps;

@@ -16,6 +16,9 @@ with each one alone and with neither:
                             the bulk variant's size threshold)
   register combine, kept slots only (capacity layouts: wide rows of a
                             skewed batch, and narrow rows)
+  staged combine (dense layouts with rows wider than 8 KiB and at least 8
+                            row slices per SM: a ring of stages per CTA; rows
+                            cut into slices, k = 16, whole rows)
 
 The sum is commutative up to fp32 rounding, so an exchange of the two
 operands' order cannot be seen at bf16 precision; what these tests catch is
@@ -54,6 +57,15 @@ CASES = [
                                        residual=True),
     Workload("capacity_narrow_shared_residual", T=3000, H=512, E=32, R=4, k=4,
              capacity_factor=1.0, zipf_s=1.2, **BOTH),
+    # staged combine (rows wider than 8 KiB): rows cut into three 4784-byte
+    # slices, the last 4768
+    Workload("ragged_slices_shared_residual", T=1200, H=7168, E=64, R=8, k=8, **BOTH),
+    # staged combine: k = 16 plus both extra rows, 18 slots of 3424 bytes a stage
+    Workload("k16_wide_shared_residual", T=600, H=5120, E=64, R=8, k=16, **BOTH),
+    # staged combine: whole 9 KiB rows, exactly 8 units per CTA
+    Workload("eight_units_per_cta_residual", T=148 * 8, H=4608, E=32, R=4, k=4, residual=True),
+    # bulk combine with k = 16 plus both extra rows
+    Workload("k16_narrow_shared_residual", T=5000, H=1024, E=64, R=8, k=16, **BOTH),
 ]
 
 
