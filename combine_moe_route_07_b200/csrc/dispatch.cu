@@ -31,28 +31,43 @@ constexpr int kThreads = 256;
 // One warp per (token, slice of 32*CPT chunks): lane l holds chunks
 // slice*32*CPT + l + 32*i, so each warp load or store is one contiguous 512 B
 // run.  Lane j < k fetches dst_pos[t][j] once; the rows are broadcast by shuffle.
+// x_ready (the fused steps 1-4, behind this library's layout kernel): x is
+// complete, so the first task's rows are loaded before waiting for dst_pos.
 template <int CPT>
 __global__ void __launch_bounds__(kThreads)
     dispatch_bf16_kernel(const char* __restrict__ x, const int32_t* __restrict__ dst_pos, int T,
-                         int H, int k, int64_t N, char* __restrict__ out, WsHeader* hdr) {
-  pdl_wait();  // x and dst_pos may come from the kernel launched just before
-  pdl_trigger();
+                         int H, int k, int64_t N, char* __restrict__ out, WsHeader* hdr,
+                         int x_ready) {
   const int lane = threadIdx.x & 31;
   const int C8 = H >> 3;  // 16-byte chunks per row
   const int S = (C8 + 32 * CPT - 1) / (32 * CPT);
   const int64_t tasks = (int64_t)T * S;
   const size_t row_bytes = (size_t)H * 2;
   const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
-  for (int64_t task = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5; task < tasks;
-       task += nw) {
+  const int64_t task0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+  auto load_rows = [&](int64_t task, uint4 (&v)[CPT]) {
     const int t = (int)((uint32_t)task / (uint32_t)S);  // tasks < 2^31 (host check)
     const int cb = (int)((uint32_t)task - (uint32_t)t * (uint32_t)S) * 32 * CPT + lane;
     const char* src = x + (size_t)t * row_bytes;
-    uint4 v[CPT];
 #pragma unroll
     for (int i = 0; i < CPT; ++i) {
       const int c = cb + 32 * i;
       if (c < C8) v[i] = ld16_stream(src + (size_t)c * 16);
+    }
+  };
+  uint4 v0[CPT];
+  if (x_ready && task0 < tasks) load_rows(task0, v0);
+  pdl_wait();  // dst_pos (and, unless x_ready, x) may come from the kernel launched just before
+  pdl_trigger();
+  for (int64_t task = task0; task < tasks; task += nw) {
+    const int t = (int)((uint32_t)task / (uint32_t)S);
+    const int cb = (int)((uint32_t)task - (uint32_t)t * (uint32_t)S) * 32 * CPT + lane;
+    uint4 v[CPT];
+    if (x_ready && task == task0) {
+#pragma unroll
+      for (int i = 0; i < CPT; ++i) v[i] = v0[i];
+    } else {
+      load_rows(task, v);
     }
     const int pl = lane < k ? __ldg(dst_pos + (size_t)t * k + lane) : -1;
     for (int j = 0; j < k; ++j) {
@@ -440,11 +455,13 @@ cudaError_t launch_dispatch_bf16(const LaunchEnv& env, const void* x, const int3
   if (C8 >= 256) {
     auto kern = dispatch_bf16_kernel<2>;
     const int grid = grid_for(kern, env, (int64_t)T * ((C8 + 63) / 64) * 32);
-    return launch_pdl(env, kern, dim3(grid), dim3(kThreads), 0, xs, dst_pos, T, H, k, N, o, hdr);
+    return launch_pdl(env, kern, dim3(grid), dim3(kThreads), 0, xs, dst_pos, T, H, k, N, o, hdr,
+                      x_ready ? 1 : 0);
   } else {
     auto kern = dispatch_bf16_kernel<1>;
     const int grid = grid_for(kern, env, (int64_t)T * ((C8 + 31) / 32) * 32);
-    return launch_pdl(env, kern, dim3(grid), dim3(kThreads), 0, xs, dst_pos, T, H, k, N, o, hdr);
+    return launch_pdl(env, kern, dim3(grid), dim3(kThreads), 0, xs, dst_pos, T, H, k, N, o, hdr,
+                      x_ready ? 1 : 0);
   }
 }
 
