@@ -187,6 +187,12 @@ def oracle_chunk(w: Workload, x_bits, ids, gates, dst_pos, tokens, shared_bits=N
         sh = shared_bits[tokens]
     res = {"keep": keep, "dispatch": disp}
     res.update(oracle_combines(y, local, gates[tokens], n, sh, xs if w.residual else None))
+    if w.fp8:  # the same combine over the unquantised rows, and the recipe's error bound
+        y16 = oracle.dispatch_bf16(xs, local, n * k)
+        res["out_unquantised"] = oracle.combine(y16, local, gates[tokens], n, shared_bits=sh,
+                                                residual_bits=xs if w.residual else None)
+        amax = np.abs(bf16_value(xs)).reshape(n, -1, 128).max(axis=2)
+        res["fp8_bound"] = np.repeat(amax, 128, axis=1) * (16.0 / 448.0)
     return res
 
 

@@ -313,3 +313,44 @@ def test_combine_f32_identity_experts_return_the_input_exactly():
     y = oracle.dispatch_bf16(x, L["dst_pos"], T * k)
     out = oracle.combine_f32(y, L["dst_pos"], gates, T)
     assert np.array_equal(_bits_to_f64(out), _bits_to_f64(x))
+
+
+def test_fp8_recipe_error_reaches_16_of_448_of_the_block_max():
+    """The FP8 recipe (per-128-channel scale = amax/448, e4m3 round to nearest
+    even) can be off by half an e4m3 step of the top binade: 16/448 (3.57 %)
+    of the block's max.  Worked by hand: a block whose max is 448 (scale 1)
+    holding 432, the midpoint of the e4m3 values 416 (mantissa 101) and 448
+    (mantissa 110), which rounds to the even 448.  Where that block holds the
+    tensor's largest value, the error is 3.57 % of max|x| -- above a 2 % of
+    max|x| bound against the unquantised rows, which no encoding with these
+    scales can meet; the FP8 path is therefore checked against the quantised
+    oracle, and against the unquantised rows within this bound."""
+    row = np.zeros(128, np.float32)
+    row[0], row[1] = 448.0, 432.0
+    xb = bf16_bits(torch.from_numpy(row).to(torch.bfloat16))
+    q, s = oracle.quantize_row_fp8(xb)
+    assert s[0] == np.float32(1.0)
+    deq = _bits_to_f64(oracle.dequant_fp8(q[None, :], s[None, :]))[0]
+    assert deq[0] == 448.0 and deq[1] == 448.0
+    err = abs(deq[1] - 432.0)
+    assert err == 16.0 and err / 448.0 > 0.035
+
+
+def test_fp8_path_within_the_recipe_bound_of_the_unquantised_combine():
+    """Identity experts behind the FP8 dispatch: every output is within
+    16/448 of its 128-channel block's max (the recipe's rounding) plus one
+    bf16 quantum of the unquantised path's output."""
+    rng = np.random.default_rng(46)
+    T, H, E, R, k = 120, 512, 32, 4, 6
+    x = _bf16_rand((T, H), rng, scale=2.0)
+    ids, gates = oracle.route(rng.standard_normal((T, E)).astype(np.float32), k)
+    L = oracle.layout(ids, E, R)
+    q, s = oracle.dispatch_fp8(x, L["dst_pos"], T * k)
+    y8 = oracle.dequant_fp8(q, s)
+    y16 = oracle.dispatch_bf16(x, L["dst_pos"], T * k)
+    a = _bits_to_f64(oracle.combine(y8, L["dst_pos"], gates, T, residual_bits=x))
+    b = _bits_to_f64(oracle.combine(y16, L["dst_pos"], gates, T, residual_bits=x))
+    amax = np.abs(_bits_to_f64(x)).reshape(T, H // 128, 128).max(axis=2)
+    bound = np.repeat(amax, 128, axis=1) * 16.0 / 448.0
+    quantum = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(b), 2.0 ** -126))) - 7)
+    assert np.all(np.abs(a - b) <= bound + quantum)
