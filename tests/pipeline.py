@@ -191,8 +191,10 @@ def oracle_chunk(w: Workload, x_bits, ids, gates, dst_pos, tokens, shared_bits=N
         y16 = oracle.dispatch_bf16(xs, local, n * k)
         res["out_unquantised"] = oracle.combine(y16, local, gates[tokens], n, shared_bits=sh,
                                                 residual_bits=xs if w.residual else None)
-        amax = np.abs(bf16_value(xs)).reshape(n, -1, 128).max(axis=2)
-        res["fp8_bound"] = np.repeat(amax, 128, axis=1) * (16.0 / 448.0)
+        # e4m3 rounding of the scaled value (16/448 of the block's max at worst),
+        # plus the bf16 rounding of the dequantised row (half a quantum of it)
+        amax = np.repeat(np.abs(bf16_value(xs)).reshape(n, -1, 128).max(axis=2), 128, axis=1)
+        res["fp8_bound"] = amax * (16.0 / 448.0) + bf16_quantum(amax)
     return res
 
 
