@@ -191,14 +191,40 @@ def small_route_layout(T, E, k):
     return T > 0 and E <= 512 and T * k <= 1024
 
 
-def kernels_per_step(path, separate, src, small, bias_update):
+# the library's limits for placing and dispatching in one kernel behind the
+# route kernel (kernels.h: kPdMinTokens; place_dispatch.cu: the pipelines, the
+# stages and the shared-memory budget)
+PD_MIN_TOKENS, PD_WARPS, PD_PIPES, PD_MAX_STAGES, PD_SMEM = 2048, 16, 4, 8, 200 * 1024
+PD_MAX_ASSIGN = 512
+
+
+def place_dispatch_one_kernel(T, E, k, H, fp8, capacity, num_sms):
+    """Whether moe_route_layout_dispatch places and dispatches in one kernel
+    (bf16 rows of 1-32 KiB, dropless, at least PD_MIN_TOKENS tokens, at most
+    PD_MAX_ASSIGN assignments a CTA, within the shared-memory budget)."""
+    row = 2 * H
+    if fp8 or capacity > 0 or T < PD_MIN_TOKENS or row < 1024 or row > 32768:
+        return False
+    TB = -(-T // num_sms)
+    if TB * k > PD_MAX_ASSIGN:
+        return False
+    ints = (PD_WARPS * E + 4 * E + 1 + 2 * TB * k) * 4
+    if ints >= PD_SMEM:
+        return False
+    return min(PD_MAX_STAGES, (PD_SMEM - ints) // (PD_PIPES * row)) >= 2
+
+
+def kernels_per_step(path, separate, src, small, bias_update, place_dispatch=False):
     """Kernels one step launches: route (1) + layout (count and place: 2; the
     per-source-rank layout 4) + dispatch + combine on the separate calls; the
-    fused paths route and lay out in 2 kernels, or 1 for a small batch."""
+    fused paths route and lay out in 2 kernels, or 1 for a small batch; the
+    fused steps 1-4 place and dispatch in one kernel when the batch fits."""
     if separate:
         n = 1 + (4 if src else 2) + 2
     elif path == "separate":
         n = 5
+    elif path == "fused3" and place_dispatch:
+        n = 3
     else:
         n = (1 if small else 2) + 2
     return n + (1 if bias_update else 0)
@@ -916,9 +942,12 @@ def main():
                      "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
                      "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
                      "traffic": ncu_traffic(dom, w.name)},
-        "gpu_launches": kernels_per_step(args.path, path.separate, path.src,
-                                         small_route_layout(T, w.E, k),
-                                         args.bias_gamma > 0) * K,
+        "gpu_launches": kernels_per_step(
+            args.path, path.separate, path.src, small_route_layout(T, w.E, k),
+            args.bias_gamma > 0,
+            place_dispatch_one_kernel(T, w.E, k, w.H, w.fp8, path.shape.capacity,
+                                      torch.cuda.get_device_properties(dev).multi_processor_count)
+        ) * K,
         "clocks": clocks,
         "e2e": e2e,
     }

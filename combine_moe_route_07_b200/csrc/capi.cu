@@ -256,10 +256,16 @@ moe_status_t moe_layout_src(const moe_shape_t* shape, const int32_t* ids, int32_
                                           src_idx));
 }
 
-moe_status_t moe_route_layout(const moe_shape_t* shape, const float* logits, const float* bias,
-                              int32_t* ids, float* gates, int32_t* counts, int32_t* expert_off,
-                              int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
-                              int32_t* src_idx, void* ws, size_t ws_bytes, moe_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The argument checks of moe_route_layout (and of the route and layout part of
+// moe_route_layout_dispatch).
+moe_status_t route_layout_args_ok(const moe_shape_t* shape, const float* logits, const float* bias,
+                                  int32_t* ids, float* gates, int32_t* counts,
+                                  int32_t* expert_off, int32_t* rank_off, int32_t* rank_counts,
+                                  int32_t* dst_pos, int32_t* src_idx, void* ws, size_t ws_bytes) {
   if (!shape_ok(shape) || src_layout(shape)) return MOE_ERR_INVALID_ARG;
   const int64_t N = rows_of(shape);
   if (counts == nullptr || expert_off == nullptr || rank_off == nullptr ||
@@ -273,8 +279,22 @@ moe_status_t moe_route_layout(const moe_shape_t* shape, const float* logits, con
                         dst_pos, src_idx};
   for (const void* p : ptrs)
     if (!aligned(p, 4)) return MOE_ERR_INVALID_ARG;
-  moe_status_t st = ws_ok(shape, ws, ws_bytes);
+  return ws_ok(shape, ws, ws_bytes);
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_route_layout(const moe_shape_t* shape, const float* logits, const float* bias,
+                              int32_t* ids, float* gates, int32_t* counts, int32_t* expert_off,
+                              int32_t* rank_off, int32_t* rank_counts, int32_t* dst_pos,
+                              int32_t* src_idx, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  const moe_status_t st = route_layout_args_ok(shape, logits, bias, ids, gates, counts,
+                                               expert_off, rank_off, rank_counts, dst_pos,
+                                               src_idx, ws, ws_bytes);
   if (st != MOE_OK) return st;
+  const int64_t N = rows_of(shape);
   WsHeader* hdr = static_cast<WsHeader*>(ws);
   uint32_t* tables = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + kHeaderBytes);
   const size_t half = half_words_of(ws_bytes);
@@ -307,6 +327,27 @@ moe_status_t moe_route_layout_dispatch(const moe_shape_t* shape, const float* lo
   if (shape->tokens > 0 && (x == nullptr || out == nullptr || (fp8 && scales == nullptr)))
     return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(out, 16) || !aligned(scales, 4)) return MOE_ERR_INVALID_ARG;
+  const int T = shape->tokens, E = shape->experts, k = shape->k, H = shape->hidden;
+  if (!fp8 && T > 0 && !moe::route_layout_small_fits(T, E, k)) {
+    const moe::LaunchEnv env = env_of(stream);
+    if (moe::place_dispatch_fits(T, E, k, H, shape->capacity, env.num_sms)) {
+      // the route kernel fills the tile table; one kernel places and streams the rows
+      const moe_status_t sa = route_layout_args_ok(shape, logits, bias, ids, gates, counts,
+                                                   expert_off, rank_off, rank_counts, dst_pos,
+                                                   src_idx, ws, ws_bytes);
+      if (sa != MOE_OK) return sa;
+      WsHeader* hdr = static_cast<WsHeader*>(ws);
+      uint32_t* tables = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + kHeaderBytes);
+      const size_t half = half_words_of(ws_bytes);
+      const cudaError_t err =
+          moe::launch_route(env, logits, bias, T, E, k, (shape->flags & MOE_F_RENORM) ? 1 : 0,
+                            ids, gates, hdr, tables, half);
+      if (err != cudaSuccess) return MOE_ERR_CUDA;
+      return from_cuda(moe::launch_place_dispatch(
+          env, ids, x, T, H, E, k, shape->ranks, shape->align, rows_of(shape), tables, half, hdr,
+          counts, expert_off, rank_off, rank_counts, dst_pos, src_idx, out));
+    }
+  }
   moe_status_t st = moe_route_layout(shape, logits, bias, ids, gates, counts, expert_off,
                                      rank_off, rank_counts, dst_pos, src_idx, ws, ws_bytes,
                                      stream);

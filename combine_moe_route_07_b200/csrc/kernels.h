@@ -161,6 +161,21 @@ cudaError_t launch_route_layout_small(const LaunchEnv& env, const float* logits,
                                       int32_t* expert_off, int32_t* rank_off,
                                       int32_t* rank_counts, int32_t* dst_pos, int32_t* src_idx);
 
+// Steps 3-4 behind a route launch with the tile table (the fused steps 1-4,
+// bf16, dropless, at least kPdMinTokens tokens, rows of 1-32 KiB, at most 512
+// assignments a CTA): each CTA
+// places a contiguous range of tokens from the tile table and streams their
+// rows by bulk copy.  Same results as launch_layout (count_ids = false) +
+// launch_dispatch_bf16.  place_dispatch_fits says whether a batch fits.
+constexpr int kPdMinTokens = 2048;
+bool place_dispatch_fits(int T, int E, int k, int H, int capacity, int num_sms);
+cudaError_t launch_place_dispatch(const LaunchEnv& env, const int32_t* ids, const void* x, int T,
+                                  int H, int E, int k, int R, int align, int64_t N,
+                                  uint32_t* tables, size_t half_words, WsHeader* hdr,
+                                  int32_t* counts, int32_t* expert_off, int32_t* rank_off,
+                                  int32_t* rank_counts, int32_t* dst_pos, int32_t* src_idx,
+                                  void* out);
+
 // Round-robin router (diagnostic): ids[t,j] = (t*k + j) mod E, gates 1/k.
 cudaError_t launch_route_round_robin(const LaunchEnv& env, int T, int E, int k, int32_t* ids,
                                      float* gates);

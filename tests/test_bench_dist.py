@@ -136,3 +136,26 @@ def test_small_route_layout_rule_matches_the_library_constants():
     assert bench.kernels_per_step("fused3", False, False, False, True) == 5
     assert bench.kernels_per_step("separate", False, False, True, False) == 5
     assert bench.kernels_per_step("fused3", True, True, False, False) == 7
+    assert bench.kernels_per_step("fused3", False, False, False, False, True) == 3
+    assert bench.kernels_per_step("fused", False, False, False, False, True) == 4
+
+
+def test_place_dispatch_rule_matches_the_library_constants():
+    """The bench's copy of the place-and-dispatch kernel's limits equals the
+    library's constants, and the rule picks the workloads it should."""
+    import re
+    import bench
+    from combine_moe_route_07_b200.workloads import WORKLOADS
+    hdr = open(os.path.join(ROOT, "combine_moe_route_07_b200", "csrc", "kernels.h")).read()
+    src = open(os.path.join(ROOT, "combine_moe_route_07_b200", "csrc", "place_dispatch.cu")).read()
+    const = lambda text, name: int(re.search(name + r" = (\d+)", text).group(1))  # noqa: E731
+    assert bench.PD_MIN_TOKENS == const(hdr, "kPdMinTokens")
+    assert bench.PD_PIPES == const(src, "kPdPipes")
+    assert bench.PD_MAX_STAGES == const(src, "kPdMaxStages")
+    assert bench.PD_WARPS * 32 == const(src, "kPdThreads")
+    assert bench.PD_SMEM == const(src, "kPdSmemBudget") * 1024
+    assert bench.PD_MAX_ASSIGN == const(src, "kPdMaxAssign")
+    fits = {n: bench.place_dispatch_one_kernel(w.T, w.E, w.k, w.H, w.fp8, w.capacity, 148)
+            for n, w in WORKLOADS.items()}
+    assert fits == {"tiny": False, "prefill": True, "decode": False, "skewed_capacity": False,
+                    "skewed_dropless": False, "finegrained": False}
