@@ -924,7 +924,8 @@ def main():
         "dispatch_combine": {"tokens_per_s": world * T / ((t_disp + t_comb) * 1e-3), **dc,
                              "method": (f"in the step: a replay of the step with event records "
                                         f"between its kernels (no launch overlap across them), "
-                                        f"mean of {K_ops}")},
+                                        f"mean of {K_ops}; a fused steps 1-4 call is timed as "
+                                        f"moe_route_layout then moe_dispatch")},
         "copy_anchor": {
             "bytes_moved": 2 * copy_bytes, "us": round(copy_ms * 1e3, 2),
             "gbs": round(2 * copy_bytes / (copy_ms * 1e-3) / 1e9, 1),
