@@ -13,7 +13,8 @@
 // STAGE (many experts per token, rows of 16-byte multiples): each warp keeps
 // two shared-memory row buffers and prefetches the logits of its next token by
 // bulk copy (TMA) while it routes the current one, so the row's DRAM latency
-// overlaps the selection arithmetic.
+// overlaps the selection arithmetic.  Without a rank limit the staged rows go
+// through route_token_fast (float keys, exact fallback to the code form).
 #include "bulk.cuh"
 #include "common.cuh"
 #include "kernels.h"
@@ -28,7 +29,7 @@ constexpr int kWarps = kThreads / 32;  // tokens per CTA group
 constexpr uint64_t kRowTimeoutNs = 1000000000ull;
 
 template <int NK, bool HIST, bool STAGE, bool LIMIT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, (STAGE && !LIMIT && NK <= 16) ? 4 : 1)
     route_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E,
                  int k, int renorm, int32_t* __restrict__ ids, float* __restrict__ gates,
                  WsHeader* hdr, uint32_t* __restrict__ tables, int TT, size_t table_words,
@@ -61,6 +62,8 @@ __global__ void __launch_bounds__(kThreads)
   pdl_trigger();
   float b[NK];
   if constexpr (!STAGE) load_bias<NK>(bias, E, lane, b);
+  FastLanes<STAGE ? NK : 8> fast;  // the staged form without a rank limit
+  if constexpr (STAGE && !LIMIT) fast.init(E, lane);
   if constexpr (STAGE) {  // the bias, read per token from shared memory
     for (int e = threadIdx.x; e < E; e += kThreads) sbias[e] = bias != nullptr ? __ldg(bias + e) : 0.0f;
     __syncthreads();
@@ -69,13 +72,14 @@ __global__ void __launch_bounds__(kThreads)
   const int c1 = min(T, c0 + per);
   const int n = (c1 - c0 + kWarps - 1) / kWarps;  // groups: the same for every warp
   uint32_t* tab = nullptr;
-  int cur_tile = 0;
+  int cur_tile = 0, tile_end = 0;  // the current tile and its first token past the end
   if constexpr (HIST) {
     const uint32_t epoch = *reinterpret_cast<volatile uint32_t*>(&hdr->epoch);
     tab = tables + (size_t)(epoch & 1u) * table_words;
     for (int e = threadIdx.x; e < E; e += kThreads) hist[e] = 0;
     __syncthreads();
     cur_tile = c0 / TT;
+    tile_end = (cur_tile + 1) * TT;
   }
   auto flush = [&](int tile) {  // caller: __syncthreads() before and after
     uint32_t* row = tab + (size_t)tile * E;
@@ -102,12 +106,12 @@ __global__ void __launch_bounds__(kThreads)
   for (int i = 0; i < n; ++i) {
     const int g0 = c0 + kWarps * i;
     if constexpr (HIST) {
-      const int tile = g0 / TT;
-      if (tile != cur_tile) {
+      if (g0 >= tile_end) {  // (the same for every warp of the CTA)
         __syncthreads();
         flush(cur_tile);
         __syncthreads();
-        cur_tile = tile;
+        cur_tile = g0 / TT;
+        tile_end = (cur_tile + 1) * TT;
       }
     }
     const int t = g0 + w;
@@ -124,8 +128,12 @@ __global__ void __launch_bounds__(kThreads)
         if (ok) {
           parity ^= 1u << sb;
           pending &= ~(1u << sb);
-          nan_tok = route_token_smem<NK, LIMIT>(buf + (size_t)sb * E, sbias, t, E, k, renorm,
-                                                lane, cand_all[w], e1, g1, lim);
+          if constexpr (LIMIT)
+            nan_tok = route_token_smem<NK, true>(buf + (size_t)sb * E, sbias, t, E, k, renorm,
+                                                 lane, cand_all[w], e1, g1, lim);
+          else
+            nan_tok = route_token_fast<NK>(buf + (size_t)sb * E, sbias, bias != nullptr, t, E,
+                                           k, renorm, lane, cand_all[w], fast, e1, g1);
         } else {
           if (lane == 0) report(hdr, MOE_ERR_DEVICE_TIMEOUT, t);
           alive = false;  // routes nothing more; still takes part in the CTA barriers

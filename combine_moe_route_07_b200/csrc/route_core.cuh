@@ -631,4 +631,192 @@ __device__ __forceinline__ int route_token_smem(const float* srow, const float* 
   return nan_tok;
 }
 
+// ---------------------------------------------------------------------------
+// The fast form for staged rows without a rank limit: the same top-k, decided
+// on the float keys themselves.  Lane l holds experts l, l+32, l+64, ... (so
+// experts with neighbouring ids, which a skewed router often makes the
+// popular ones, sit on different lanes and tau stays tight).  Float order is
+// the key order here: +0 and -0 compare equal, as their folded codes do, and
+// NaN is excluded up front.
+//   1. lane maximum by three-input max.NaN: a NaN key makes it NaN, and one
+//      NaN-propagating warp max per token then detects any NaN key;
+//   2. tau = the k-th largest lane maximum (k rounds of a float warp max);
+//   3. the keys >= tau (k to k+4 typically, at most 32 taken here) are
+//      compacted by ballot rounds into shared memory as (value, expert);
+//   4. candidate i's slot is the number of candidates with a strictly larger
+//      value, read four at a time; with no two equal values that is the
+//      exact order, and two equal values among the first k slots land on the
+//      same slot, which the writer check below detects.
+// A NaN key, more than 32 candidates or equal values at a slot below k take
+// the exact code-based form (route_token_smem), so every result is the same
+// bits as that form's.
+constexpr int kFastMaxCand = 32;
+
+__device__ __forceinline__ float max3_nan(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float max2_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+__device__ __forceinline__ float warp_max_nan(float v) {
+  float r;
+  asm volatile("redux.sync.max.NaN.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+__device__ __forceinline__ float warp_max_redux(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
+// Per-lane constant: bit i is set when key i (expert lane + 32 i) is < E.
+template <int NK>
+struct FastLanes {
+  uint32_t vmask = 0u;
+  __device__ void init(int E, int lane) {
+    vmask = 0u;
+#pragma unroll
+    for (int i = 0; i < NK; ++i)
+      if (lane + 32 * i < E) vmask |= 1u << i;
+  }
+};
+
+// Selection only: true with lane j < k holding slot j's expert and raw logit,
+// false when the token needs the exact form (nothing is decided then).
+template <int NK>
+__device__ __forceinline__ bool select_fast(const float* srow, const float* sbias, bool has_bias,
+                                            int k, int lane, uint32_t* cand,
+                                            const FastLanes<NK>& F, int& sel_e,
+                                            float& sel_raw) {
+  static_assert(NK >= 8 && NK <= 32, "the staged form");
+  float key[NK];
+  if (has_bias) {
+#pragma unroll
+    for (int i = 0; i < NK; ++i) {
+      const int e = lane + 32 * i;
+      key[i] = ((F.vmask >> i) & 1u) ? __fadd_rn(srow[e], sbias[e]) : -INFINITY;
+    }
+  } else if (F.vmask == (NK == 32 ? 0xffffffffu : (1u << NK) - 1u)) {
+#pragma unroll
+    for (int i = 0; i < NK; ++i) key[i] = srow[lane + 32 * i];
+  } else {
+#pragma unroll
+    for (int i = 0; i < NK; ++i) key[i] = ((F.vmask >> i) & 1u) ? srow[lane + 32 * i] : -INFINITY;
+  }
+  // 1. lane maximum; any NaN key makes the warp maximum NaN
+  float mm = key[0];
+#pragma unroll
+  for (int i = 1; i + 1 < NK; i += 2) mm = max3_nan(mm, key[i], key[i + 1]);
+  mm = max2_nan(mm, key[NK - 1]);  // NK is even: the last key is left over
+  const float wmax = warp_max_nan(mm);
+  if (wmax != wmax) return false;
+  auto candidates = [&](float tau, uint32_t& cm) {
+    cm = 0u;
+#pragma unroll
+    for (int i = 0; i < NK; ++i) cm |= (key[i] >= tau) ? (1u << i) : 0u;
+    cm &= F.vmask;
+    return (int)__reduce_add_sync(kFull, (unsigned)__popc(cm));
+  };
+  // 2. tau: the k-th largest lane maximum
+  float tau = wmax;
+  {
+    float m = mm;
+#pragma unroll 1
+    for (int j = 0; j < k; ++j) {
+      const float top = warp_max_redux(m);
+      tau = top;
+      const unsigned hold = __ballot_sync(kFull, m == top);
+      if (lane == __ffs(hold) - 1) m = -INFINITY;
+    }
+  }
+  uint32_t cm = 0u;
+#pragma unroll
+  for (int i = 0; i < NK; ++i) cm |= (key[i] >= tau) ? (1u << i) : 0u;
+  cm &= F.vmask;
+  const int total = (int)__reduce_add_sync(kFull, (unsigned)__popc(cm));
+  if (total > kFastMaxCand) return false;
+  // 3. compaction by ballot rounds: (value, expert) of candidate p at cv[p], ce[p]
+  float* cv = reinterpret_cast<float*>(cand);     // kFastMaxCand + 4 words
+  int* ce = reinterpret_cast<int*>(cand + 64);     // kFastMaxCand words
+  int* slot = reinterpret_cast<int*>(cand + 128);  // k words
+  int base = 0;
+#pragma unroll 1
+  while (true) {
+    const unsigned any = __ballot_sync(kFull, cm != 0u);
+    if (any == 0u) break;
+    if (cm != 0u) {
+      const int e = lane + 32 * (__ffs(cm) - 1);
+      const int p = base + __popc(any & lanemask_lt());
+      cv[p] = has_bias ? __fadd_rn(srow[e], sbias[e]) : srow[e];
+      ce[p] = e;
+      cm &= cm - 1u;
+    }
+    base += __popc(any);
+  }
+  if (lane < 4) cv[total + lane] = -INFINITY;  // pads the last group of four
+  __syncwarp();
+  // 4. slots: candidates with a strictly larger value
+  int n = 0;
+  const float v = lane < total ? cv[lane] : INFINITY;
+#pragma unroll 1
+  for (int m0 = 0; m0 < total; m0 += 4) {
+    const float4 q = *reinterpret_cast<const float4*>(cv + m0);
+    n += (q.x > v) + (q.y > v) + (q.z > v) + (q.w > v);
+  }
+  const bool mine = lane < total && n < k;
+  if (mine) slot[n] = lane;
+  __syncwarp();
+  const bool clash = mine && slot[n] != lane;
+  if (__any_sync(kFull, clash)) {  // equal values among the first k
+    __syncwarp();
+    return false;
+  }
+  if (lane < k) {
+    sel_e = ce[slot[lane]];
+    sel_raw = srow[sel_e];
+  }
+  __syncwarp();  // the next token may overwrite the candidates
+  return true;
+}
+
+// The exact code-based form, out of line: it runs for rare tokens only, and
+// kept apart it does not raise the fast form's register count.
+template <int NK>
+__device__ __noinline__ int route_token_exact(const float* srow, const float* sbias, int t, int E,
+                                              int k, int renorm, int lane, uint32_t* cand,
+                                              int& sel_e, float& gate) {
+  return route_token_smem<NK, false>(srow, sbias, t, E, k, renorm, lane, cand, sel_e, gate,
+                                     RankLimit());
+}
+
+template <int NK>
+__device__ __forceinline__ int route_token_fast(const float* srow, const float* sbias,
+                                                bool has_bias, int t, int E, int k, int renorm,
+                                                int lane, uint32_t* cand, const FastLanes<NK>& F,
+                                                int& sel_e, float& gate) {
+  sel_e = 0;
+  float sel_raw = 0.0f;
+  if (!select_fast<NK>(srow, sbias, has_bias, k, lane, cand, F, sel_e, sel_raw))
+    return route_token_exact<NK>(srow, sbias, t, E, k, renorm, lane, cand, sel_e, gate);
+  if (renorm) {
+    const float m = warp_max_f(lane < k ? sel_raw : -INFINITY);
+    const double ex = (lane < k) ? exp((double)sel_raw - (double)m) : 0.0;
+    const double den = warp_sum_d(ex);
+    gate = (float)(ex * __drcp_rn(den));
+  } else {
+    float lm = -INFINITY;
+    for (int e = lane; e < E; e += 32) lm = fmaxf(lm, srow[e]);
+    const float m = warp_max_f(lm);
+    double part = 0.0;
+    for (int e = lane; e < E; e += 32) part += exp((double)srow[e] - (double)m);
+    const double den = warp_sum_d(part);
+    gate = (float)(exp((double)sel_raw - (double)m) * __drcp_rn(den));
+  }
+  return -1;
+}
+
 }  // namespace moe
