@@ -11,10 +11,11 @@
 // most once per tile it touches rather than once per group.
 //
 // STAGE (many experts per token, rows of 16-byte multiples): each warp keeps
-// two shared-memory row buffers and prefetches the logits of its next token by
-// bulk copy (TMA) while it routes the current one, so the row's DRAM latency
-// overlaps the selection arithmetic.  Without a rank limit the staged rows go
-// through route_token_fast (float keys, exact fallback to the code form).
+// two or three shared-memory row buffers and prefetches the logits of its
+// next one or two tokens by bulk copy (TMA) while it routes the current one,
+// so the rows' DRAM latency overlaps the selection arithmetic.  Without a rank limit the staged
+// rows go through route_token_fast (float keys, exact fallback to the code
+// form).
 #include "bulk.cuh"
 #include "common.cuh"
 #include "kernels.h"
@@ -27,6 +28,11 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;  // tokens per CTA group
 constexpr uint64_t kRowTimeoutNs = 1000000000ull;
+// STAGE: row buffers per warp.  Three (two rows in flight ahead) for rows of
+// up to 256 experts; two for longer rows, whose third buffer would cost a CTA
+// per SM (Fine-grained, 512 experts: 75 us with two against 88 with three).
+constexpr int row_stages(int nk) { return nk <= 8 ? 3 : 2; }
+constexpr int kMaxRowStages = 3;
 
 template <int NK, bool HIST, bool STAGE, bool LIMIT>
 __global__ void __launch_bounds__(kThreads, (STAGE && !LIMIT && NK <= 16) ? 4 : 1)
@@ -34,27 +40,28 @@ __global__ void __launch_bounds__(kThreads, (STAGE && !LIMIT && NK <= 16) ? 4 : 
                  int k, int renorm, int32_t* __restrict__ ids, float* __restrict__ gates,
                  WsHeader* hdr, uint32_t* __restrict__ tables, int TT, size_t table_words,
                  int per, int R, int M) {
-  // dynamic: [hist: E int32, padded to 16 B] (HIST), [rows: kWarps x 2 x E floats] (STAGE),
+  // dynamic: [hist: E int32, padded to 16 B] (HIST), [rows: kWarps x kRowStages x E floats]
+  // (STAGE),
   // [rank limit: kWarps x (R + ceil(R/32)) words] (M < R), [bias: E floats] (STAGE)
   extern __shared__ __align__(16) unsigned char dyn[];
   __shared__ __align__(16) uint32_t cand_all[kWarps][NK >= 8 ? 3 * kMaxCand : 1];
-  __shared__ uint64_t bars[kWarps][2];
+  constexpr int kRowStages = row_stages(NK);
+  __shared__ uint64_t bars[kWarps][kMaxRowStages];
   int32_t* hist = reinterpret_cast<int32_t*>(dyn);
   const size_t hist_bytes = HIST ? (((size_t)E * 4 + 15) & ~(size_t)15) : 0;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  float* buf = reinterpret_cast<float*>(dyn + hist_bytes) + (size_t)w * 2 * E;
+  float* buf = reinterpret_cast<float*>(dyn + hist_bytes) + (size_t)w * kRowStages * E;
   RankLimit lim;  // compiled in only for LIMIT (then M < R)
   lim.R = R;
   lim.M = LIMIT ? M : 0;
   lim.init(E, lane);
   const size_t lim_words = lim.on() ? (size_t)R + (R + 31) / 32 : 0;
   uint32_t* lim_base = reinterpret_cast<uint32_t*>(
-      dyn + hist_bytes + (STAGE ? (size_t)kWarps * 2 * E * sizeof(float) : 0));
+      dyn + hist_bytes + (STAGE ? (size_t)kWarps * kRowStages * E * sizeof(float) : 0));
   if (lim.on()) lim.smem = lim_base + (size_t)w * lim_words;
   float* sbias = reinterpret_cast<float*>(lim_base + (size_t)kWarps * lim_words);
   if (STAGE && lane == 0) {
-    mbar_init(&bars[w][0], 1);
-    mbar_init(&bars[w][1], 1);
+    for (int q = 0; q < kRowStages; ++q) mbar_init(&bars[w][q], 1);
     mbar_fence_init();
   }
   __syncwarp();
@@ -91,17 +98,21 @@ __global__ void __launch_bounds__(kThreads, (STAGE && !LIMIT && NK <= 16) ? 4 : 
       }
     }
   };
-  // STAGE: buffer s of this warp holds token (c0 + w + 8*i) for i of parity s
+  // STAGE: buffer i mod kRowStages of this warp holds token c0 + w + 8*i
   uint32_t parity = 0, pending = 0;
+  int sb = 0;  // the buffer of the current token
   bool alive = true;
-  auto issue = [&](int tok, int sb) {
+  auto issue = [&](int tok, int q) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(&bars[w][sb], (uint32_t)E * 4u);
-      bulk_load(buf + (size_t)sb * E, logits + (size_t)tok * E, (uint32_t)E * 4u, &bars[w][sb]);
+      mbar_arrive_expect_tx(&bars[w][q], (uint32_t)E * 4u);
+      bulk_load(buf + (size_t)q * E, logits + (size_t)tok * E, (uint32_t)E * 4u, &bars[w][q]);
     }
-    pending |= 1u << sb;
+    pending |= 1u << q;
   };
-  if (STAGE && c0 + w < c1) issue(c0 + w, 0);
+  if constexpr (STAGE) {
+    for (int q = 0; q + 1 < kRowStages; ++q)
+      if (c0 + w + kWarps * q < c1) issue(c0 + w + kWarps * q, q);
+  }
 
   for (int i = 0; i < n; ++i) {
     const int g0 = c0 + kWarps * i;
@@ -120,9 +131,10 @@ __global__ void __launch_bounds__(kThreads, (STAGE && !LIMIT && NK <= 16) ? 4 : 
       float g1 = 0.0f;
       int nan_tok;
       if constexpr (STAGE) {
-        const int sb = i & 1;
-        // the other buffer was last read for token i-1 (done: __syncwarp below)
-        if (t + kWarps < c1) issue(t + kWarps, sb ^ 1);
+        // the buffer before this one was last read for token i-1 (done:
+        // __syncwarp below); it takes token i + kRowStages - 1
+        const int ahead = t + kWarps * (kRowStages - 1);
+        if (ahead < c1) issue(ahead, sb == 0 ? kRowStages - 1 : sb - 1);
         const bool ok = __all_sync(
             kFull, mbar_wait_bounded(&bars[w][sb], (parity >> sb) & 1u, kRowTimeoutNs));
         if (ok) {
@@ -157,12 +169,15 @@ __global__ void __launch_bounds__(kThreads, (STAGE && !LIMIT && NK <= 16) ? 4 : 
         }
       }
     }
-    if constexpr (STAGE) __syncwarp();  // every lane is done with this buffer
+    if constexpr (STAGE) {
+      __syncwarp();  // every lane is done with this buffer
+      sb = sb + 1 == kRowStages ? 0 : sb + 1;
+    }
   }
   if constexpr (STAGE) {  // copies still in flight land before the CTA exits
-    for (int sb = 0; sb < 2; ++sb)
-      if ((pending >> sb) & 1u)
-        (void)mbar_wait_bounded(&bars[w][sb], (parity >> sb) & 1u, kRowTimeoutNs);
+    for (int q = 0; q < kRowStages; ++q)
+      if ((pending >> q) & 1u)
+        (void)mbar_wait_bounded(&bars[w][q], (parity >> q) & 1u, kRowTimeoutNs);
   }
   if constexpr (HIST) {
     __syncthreads();
@@ -182,7 +197,8 @@ cudaError_t launch_nk(const LaunchEnv& env, const float* logits, const float* bi
                              : route_kernel<NK, HIST, NK >= 8, false>)
                     : (limit ? route_kernel<NK, HIST, false, true>
                              : route_kernel<NK, HIST, false, false>);
-  const size_t smem = hist_bytes + (stage ? (size_t)kWarps * 2 * E * sizeof(float) : 0) +
+  const size_t smem = hist_bytes +
+                      (stage ? (size_t)kWarps * row_stages(NK) * E * sizeof(float) : 0) +
                       (limit ? (size_t)kWarps * (R + (R + 31) / 32) * sizeof(uint32_t) : 0) +
                       (stage ? (size_t)E * sizeof(float) : 0);
   int per_sm = 1;

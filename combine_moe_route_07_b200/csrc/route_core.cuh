@@ -36,6 +36,12 @@ __device__ __forceinline__ uint32_t order_code(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The float an order code stands for (the inverse of order_code on codes of
+// non-NaN floats; +0 for the code of a folded zero).
+__device__ __forceinline__ float code_float(uint32_t c) {
+  return __uint_as_float((c & 0x80000000u) ? (c & 0x7fffffffu) : ~c);
+}
+
 __device__ __forceinline__ float warp_max_f(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
@@ -640,7 +646,8 @@ __device__ __forceinline__ int route_token_smem(const float* srow, const float* 
 // NaN is excluded up front.
 //   1. lane maximum by three-input max.NaN: a NaN key makes it NaN, and one
 //      NaN-propagating warp max per token then detects any NaN key;
-//   2. tau = the k-th largest lane maximum (k rounds of a float warp max);
+//   2. tau = the k-th largest lane maximum (k rounds of an integer warp max on
+//      order codes, lowered at most to the bottom of a 32-code bucket);
 //   3. the keys >= tau (k to k+4 typically, at most 32 taken here) are
 //      compacted by ballot rounds into shared memory as (value, expert);
 //   4. candidate i's slot is the number of candidates with a strictly larger
@@ -665,11 +672,6 @@ __device__ __forceinline__ float max2_nan(float a, float b) {
 __device__ __forceinline__ float warp_max_nan(float v) {
   float r;
   asm volatile("redux.sync.max.NaN.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
-  return r;
-}
-__device__ __forceinline__ float warp_max_redux(float v) {
-  float r;
-  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
   return r;
 }
 
@@ -721,18 +723,20 @@ __device__ __forceinline__ bool select_fast(const float* srow, const float* sbia
     cm &= F.vmask;
     return (int)__reduce_add_sync(kFull, (unsigned)__popc(cm));
   };
-  // 2. tau: the k-th largest lane maximum
-  float tau = wmax;
-  {
-    float m = mm;
+  // 2. tau: the k-th largest lane maximum, taken on order codes whose low 5
+  //    bits are replaced by the lane (each code unique, so a round is one
+  //    integer warp max and the holder clears its own); the truncation can
+  //    only lower tau, to the smallest float of the truncated code, which
+  //    still has k keys at or above it
+  uint32_t m = (order_code(mm) & ~31u) | (uint32_t)(31 - lane);
+  uint32_t top = 0u;
 #pragma unroll 1
-    for (int j = 0; j < k; ++j) {
-      const float top = warp_max_redux(m);
-      tau = top;
-      const unsigned hold = __ballot_sync(kFull, m == top);
-      if (lane == __ffs(hold) - 1) m = -INFINITY;
-    }
+  for (int j = 0; j < k; ++j) {
+    top = __reduce_max_sync(kFull, m);
+    m = (m == top) ? 0u : m;
   }
+  // (codes below 2^23 are -inf, whose truncated code would read as a NaN)
+  const float tau = top < 0x00800000u ? -INFINITY : code_float(top & ~31u);
   uint32_t cm = 0u;
 #pragma unroll
   for (int i = 0; i < NK; ++i) cm |= (key[i] >= tau) ? (1u << i) : 0u;

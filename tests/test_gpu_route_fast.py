@@ -167,3 +167,41 @@ def test_candidate_counts_around_the_limits(E, k, count):
     n = (lg >= 100.5).sum(axis=1)  # the construction's count
     assert (n == count).all(), (n.min(), n.max(), count)
     _check(lg, k)
+
+
+@pytest.mark.parametrize("E,k,T", [(8, 2, 100), (128, 8, 3000), (512, 10, 3000), (256, 8, 120)])
+@pytest.mark.parametrize("renorm", [True, False])
+def test_gates_over_the_exponent_range(E, k, T, renorm):
+    """The gates' fp64 softmax over exponential arguments from 0 down past
+    -700: logits scaled by 0.01 up to 300, so the smallest gates underflow
+    in fp32.  Every route form (one-launch cluster for small T,
+    register rows for E <= 224, staged rows above) must stay within the gate
+    tolerance, and the fp32 gates must equal the oracle's (libm fp64
+    exponential, the same rounding) in all but a few cases near an fp32
+    rounding boundary."""
+    rng = np.random.default_rng(E + T + renorm)
+    scales = np.array([0.01, 1.0, 30.0, 300.0], np.float32)
+    lg = (rng.standard_normal((T, E)).astype(np.float32)
+          * scales[np.arange(T) % 4, None]).astype(np.float32)
+    ids_o, gates_o = oracle.route(lg, k, renorm=renorm)
+    for ids, gates, err in _route_both(lg, k, renorm=renorm):
+        assert err == (0, 0)
+        assert np.array_equal(ids, ids_o)
+        assert_gates_close(gates, gates_o)
+        same = (gates.view(np.uint32) == gates_o.view(np.uint32)).mean()
+        assert same >= 0.999, same
+        assert (gates_o == 0).any() == (gates == 0).any()
+
+
+@pytest.mark.parametrize("finite", [1, 5, 10, 40])
+def test_rows_with_few_finite_keys(finite):
+    """All but `finite` keys of each row are -inf, so with finite < k fewer
+    than k lanes have a finite maximum and tau is -inf (every key a
+    candidate: the exact form); the selection runs on into the -inf keys by
+    expert id and their gates are 0."""
+    rng = np.random.default_rng(finite)
+    E, k, T = 512, 10, 2000
+    lg = np.full((T, E), -np.inf, np.float32)
+    for t in range(T):
+        lg[t, rng.choice(E, size=finite, replace=False)] = rng.standard_normal(finite)
+    _check(lg, k)
