@@ -13,9 +13,10 @@
 // STAGE (many experts per token, rows of 16-byte multiples): each warp keeps
 // two or three shared-memory row buffers and prefetches the logits of its
 // next one or two tokens by bulk copy (TMA) while it routes the current one,
-// so the rows' DRAM latency overlaps the selection arithmetic.  Without a rank limit the staged
-// rows go through route_token_fast (float keys, exact fallback to the code
-// form).
+// so the rows' DRAM latency overlaps the selection arithmetic.  Without a
+// rank limit the staged rows go through select_fast (float keys, exact
+// fallback to the code form), and with renormalised gates and k <= 16 the
+// softmax of two consecutive tokens of a warp runs as one pass.
 #include "bulk.cuh"
 #include "common.cuh"
 #include "kernels.h"
@@ -113,6 +114,12 @@ __global__ void __launch_bounds__(kThreads, (STAGE && !LIMIT && NK <= 16) ? 4 : 
     for (int q = 0; q + 1 < kRowStages; ++q)
       if (c0 + w + kWarps * q < c1) issue(c0 + w + kWarps * q, q);
   }
+  // the float-key form with renormalised gates and k <= 16: a token's softmax
+  // waits for the warp's next token of that form and the two are done in one
+  // pass (the same bits as one at a time); p_t is the waiting token
+  const bool pair = STAGE && !LIMIT && renorm && k <= 16;
+  int p_t = -1;
+  float p_raw = 0.0f;
 
   for (int i = 0; i < n; ++i) {
     const int g0 = c0 + kWarps * i;
@@ -130,6 +137,7 @@ __global__ void __launch_bounds__(kThreads, (STAGE && !LIMIT && NK <= 16) ? 4 : 
       int e1 = 0;
       float g1 = 0.0f;
       int nan_tok;
+      bool gate_ready = true;  // false: the softmax waits for the next token
       if constexpr (STAGE) {
         // the buffer before this one was last read for token i-1 (done:
         // __syncwarp below); it takes token i + kRowStages - 1
@@ -140,12 +148,30 @@ __global__ void __launch_bounds__(kThreads, (STAGE && !LIMIT && NK <= 16) ? 4 : 
         if (ok) {
           parity ^= 1u << sb;
           pending &= ~(1u << sb);
-          if constexpr (LIMIT)
-            nan_tok = route_token_smem<NK, true>(buf + (size_t)sb * E, sbias, t, E, k, renorm,
-                                                 lane, cand_all[w], e1, g1, lim);
-          else
-            nan_tok = route_token_fast<NK>(buf + (size_t)sb * E, sbias, bias != nullptr, t, E,
-                                           k, renorm, lane, cand_all[w], fast, e1, g1);
+          const float* srow = buf + (size_t)sb * E;
+          if constexpr (LIMIT) {
+            nan_tok = route_token_smem<NK, true>(srow, sbias, t, E, k, renorm, lane, cand_all[w],
+                                                 e1, g1, lim);
+          } else {
+            float raw1 = 0.0f;
+            nan_tok = -1;
+            if (!select_fast<NK>(srow, sbias, bias != nullptr, k, lane, cand_all[w], fast, e1,
+                                 raw1)) {
+              nan_tok = route_token_exact<NK>(srow, sbias, t, E, k, renorm, lane, cand_all[w],
+                                              e1, g1);
+            } else if (!pair) {
+              g1 = gate_staged(srow, raw1, E, k, renorm, lane);
+            } else if (p_t < 0) {
+              p_t = t;
+              p_raw = raw1;
+              gate_ready = false;
+            } else {
+              float ga;
+              gate_renorm_pair(p_raw, raw1, k, lane, ga, g1);
+              if (lane < k) gates[(size_t)p_t * k + lane] = ga;
+              p_t = -1;
+            }
+          }
         } else {
           if (lane == 0) report(hdr, MOE_ERR_DEVICE_TIMEOUT, t);
           alive = false;  // routes nothing more; still takes part in the CTA barriers
@@ -164,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, (STAGE && !LIMIT && NK <= 16) ? 4 : 
         if (nan_tok >= 0 && lane == 0) report(hdr, MOE_ERR_DEVICE_NAN, nan_tok);
         if (lane < k) {
           ids[(size_t)t * k + lane] = e1;
-          gates[(size_t)t * k + lane] = g1;
+          if (gate_ready) gates[(size_t)t * k + lane] = g1;
           if constexpr (HIST) atomicAdd(&hist[e1], 1);
         }
       }
@@ -173,6 +199,10 @@ __global__ void __launch_bounds__(kThreads, (STAGE && !LIMIT && NK <= 16) ? 4 : 
       __syncwarp();  // every lane is done with this buffer
       sb = sb + 1 == kRowStages ? 0 : sb + 1;
     }
+  }
+  if (p_t >= 0) {  // a token whose softmax still waits: alone
+    const float g = gate_renorm(p_raw, k, lane);
+    if (lane < k) gates[(size_t)p_t * k + lane] = g;
   }
   if constexpr (STAGE) {  // copies still in flight land before the CTA exits
     for (int q = 0; q < kRowStages; ++q)

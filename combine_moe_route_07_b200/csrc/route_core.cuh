@@ -797,30 +797,50 @@ __device__ __noinline__ int route_token_exact(const float* srow, const float* sb
                                      RankLimit());
 }
 
-template <int NK>
-__device__ __forceinline__ int route_token_fast(const float* srow, const float* sbias,
-                                                bool has_bias, int t, int E, int k, int renorm,
-                                                int lane, uint32_t* cand, const FastLanes<NK>& F,
-                                                int& sel_e, float& gate) {
-  sel_e = 0;
-  float sel_raw = 0.0f;
-  if (!select_fast<NK>(srow, sbias, has_bias, k, lane, cand, F, sel_e, sel_raw))
-    return route_token_exact<NK>(srow, sbias, t, E, k, renorm, lane, cand, sel_e, gate);
-  if (renorm) {
-    const float m = warp_max_f(lane < k ? sel_raw : -INFINITY);
-    const double ex = (lane < k) ? exp((double)sel_raw - (double)m) : 0.0;
-    const double den = warp_sum_d(ex);
-    gate = (float)(ex * __drcp_rn(den));
-  } else {
-    float lm = -INFINITY;
-    for (int e = lane; e < E; e += 32) lm = fmaxf(lm, srow[e]);
-    const float m = warp_max_f(lm);
-    double part = 0.0;
-    for (int e = lane; e < E; e += 32) part += exp((double)srow[e] - (double)m);
-    const double den = warp_sum_d(part);
-    gate = (float)(exp((double)sel_raw - (double)m) * __drcp_rn(den));
-  }
-  return -1;
+// Renormalised gates of one token whose slot j (j < k) sits on lane j: the
+// softmax of the selected raw logits, as in the forms above.
+__device__ __forceinline__ float gate_renorm(float sel_raw, int k, int lane) {
+  const float m = warp_max_f(lane < k ? sel_raw : -INFINITY);
+  const double ex = (lane < k) ? exp((double)sel_raw - (double)m) : 0.0;
+  const double den = warp_sum_d(ex);
+  return (float)(ex * __drcp_rn(den));
+}
+
+// The same for two tokens at once (k <= 16): token A's slots on lanes 0..15,
+// token B's moved to lanes 16..31, each half reduced on its own, so one pass
+// of the fp64 exponential and reciprocal serves both.  For k <= 16 the
+// one-token form's first reduction step (across the halves) only adds zeros
+// and -inf, so both give the same bits.  On return lane j < k holds A's slot
+// j gate in ga and B's in gb.
+__device__ __forceinline__ void gate_renorm_pair(float ra, float rb, int k, int lane, float& ga,
+                                                 float& gb) {
+  const float rb_hi = __shfl_sync(kFull, rb, lane & 15);
+  const float x = lane < 16 ? ra : rb_hi;
+  const bool act = (lane & 15) < k;
+  float m = act ? x : -INFINITY;
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+  const double ex = act ? exp((double)x - (double)m) : 0.0;
+  double den = ex;
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) den += __shfl_xor_sync(kFull, den, o);
+  const float g = (float)(ex * __drcp_rn(den));
+  ga = g;
+  gb = __shfl_sync(kFull, g, (lane + 16) & 31);
+}
+
+// Gates of one token from the staged row (renorm: the selected logits only;
+// else the softmax over all E logits read at the selected experts).
+__device__ __forceinline__ float gate_staged(const float* srow, float sel_raw, int E, int k,
+                                             int renorm, int lane) {
+  if (renorm) return gate_renorm(sel_raw, k, lane);
+  float lm = -INFINITY;
+  for (int e = lane; e < E; e += 32) lm = fmaxf(lm, srow[e]);
+  const float m = warp_max_f(lm);
+  double part = 0.0;
+  for (int e = lane; e < E; e += 32) part += exp((double)srow[e] - (double)m);
+  const double den = warp_sum_d(part);
+  return (float)(exp((double)sel_raw - (double)m) * __drcp_rn(den));
 }
 
 }  // namespace moe
