@@ -8,11 +8,13 @@
 // Lane l holds experts l, l+32, l+64, ... of each token in registers, as
 // order-preserving 32-bit codes of key = logit + bias.  Each of the k rounds
 // is two hardware warp reductions (redux.sync): the largest code, then the
-// lowest expert id among the lanes holding it, which is the tie rule.  Three
+// lowest expert id among the lanes holding it, which is the tie rule.  Four
 // forms of the same selection: route_tokens (every code, k rounds; E <= 224),
 // route_token_thr (a threshold first, then the few keys above it ranked
-// against each other) and route_token_smem (the threshold form with the row and the
-// bias read from shared memory, only the codes in registers).  An optional
+// against each other), route_token_smem (the threshold form with the row and
+// the bias read from shared memory, only the codes in registers) and
+// select_fast (the threshold form on the float keys of a staged row, which
+// hands ties, NaN and large candidate sets to route_token_smem).  An optional
 // rank limit clears the codes of all but the M best ranks first.  The gates
 // are a softmax of the selected RAW logits evaluated in fp64 (k values per
 // token): fp64 exponentials and sum, the quotient as the exponential times the
@@ -716,13 +718,6 @@ __device__ __forceinline__ bool select_fast(const float* srow, const float* sbia
   mm = max2_nan(mm, key[NK - 1]);  // NK is even: the last key is left over
   const float wmax = warp_max_nan(mm);
   if (wmax != wmax) return false;
-  auto candidates = [&](float tau, uint32_t& cm) {
-    cm = 0u;
-#pragma unroll
-    for (int i = 0; i < NK; ++i) cm |= (key[i] >= tau) ? (1u << i) : 0u;
-    cm &= F.vmask;
-    return (int)__reduce_add_sync(kFull, (unsigned)__popc(cm));
-  };
   // 2. tau: the k-th largest lane maximum, taken on order codes whose low 5
   //    bits are replaced by the lane (each code unique, so a round is one
   //    integer warp max and the holder clears its own); the truncation can
